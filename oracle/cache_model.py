@@ -1,0 +1,49 @@
+"""Oracle model of the cache contents -- TEST INFRASTRUCTURE ONLY.
+
+Host numpy pools laid out [num_layers][num_blocks][num_kv_heads][block_size][head_dim]
+(storage dtype: float32 / float16 / uint16 bit patterns for bf16), written the
+way the pages describe:
+
+* "What problem does PagedAttention solve, and what is continuous batching?",
+  section "Why the KV cache becomes the problem": each decode step reads the
+  cache and appends a small amount of new data -- the new token's key and value
+  rows go into the slot the block manager handed out (slot = block * B + offset).
+* same page, section "How PagedAttention works": copy-on-write gives a diverging
+  sequence a private copy of the shared block; the copy here is the whole block,
+  every layer, keys and values (a reading: the pages do not say how much is
+  copied, and copying the whole block keeps every earlier slot valid).
+
+Writes are bit copies, so the GPU pools must match these arrays exactly.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from synthetic.values import ELEM_BYTES
+
+_NP = {"f32": np.float32, "f16": np.float16, "bf16": np.uint16}
+
+
+def empty_pools(num_layers, num_blocks, num_kv_heads, block_size, head_dim, dtype):
+    shape = (num_layers, num_blocks, num_kv_heads, block_size, head_dim)
+    assert ELEM_BYTES[dtype] == np.dtype(_NP[dtype]).itemsize
+    return np.zeros(shape, _NP[dtype]), np.zeros(shape, _NP[dtype])
+
+
+def append_rows(k_pool, v_pool, layer, slots, k_rows, v_rows):
+    """Write row i of k_rows / v_rows ([n][Hkv][d]) into slot slots[i] of ``layer``."""
+    block_size = k_pool.shape[3]
+    for i, slot in enumerate(slots):
+        slot = int(slot)
+        if slot < 0:
+            continue                       # padding row: nothing is written
+        blk, off = divmod(slot, block_size)
+        k_pool[layer, blk, :, off, :] = k_rows[i]
+        v_pool[layer, blk, :, off, :] = v_rows[i]
+
+
+def copy_blocks(k_pool, v_pool, pairs):
+    """Copy-on-write: physical block dst becomes a copy of src in every layer, K and V."""
+    for src, dst in pairs:
+        k_pool[:, int(dst)] = k_pool[:, int(src)]
+        v_pool[:, int(dst)] = v_pool[:, int(src)]

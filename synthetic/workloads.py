@@ -1,0 +1,112 @@
+"""Seeded workload recipes for the five decode workloads (host side).
+
+Holds only random draws and sizes: sequence lengths, the shuffled order of the
+physical block pool, stop draws of the continuous batch, prefix/suffix lengths.
+Nothing here allocates blocks or computes attention; both the GPU path and the
+oracle consume these recipes.  Every draw comes from
+``numpy.random.default_rng(seed)`` with seed = workload number (1..5) unless a
+caller passes another.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+
+@dataclass
+class Shape:
+    """Cache geometry of one workload."""
+    num_layers: int
+    block_size: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    dtype: str            # "f32" | "f16" | "bf16"
+    num_blocks: int
+    kv_scale: float       # standard deviation of synthetic K and V values
+    q_scale: float = 1.0  # standard deviation of synthetic q values
+
+
+def tiny(seed: int = 1) -> dict:
+    """4 sequences of 50/17/3/33 tokens, block 16, 4 q / 2 KV heads, d64, fp32, 64-block pool."""
+    rng = np.random.default_rng(seed)
+    shape = Shape(1, 16, 4, 2, 64, "f32", 64, kv_scale=1.0)
+    return dict(name="tiny", seed=seed, shape=shape, lens=np.array([50, 17, 3, 33]),
+                order=rng.permutation(shape.num_blocks).astype(np.int32))
+
+
+def worked_example(seed: int = 2) -> dict:
+    """The pages' four requests (3900/420/2100/70 tokens), 32 q / 8 KV heads, d128, fp16."""
+    rng = np.random.default_rng(seed)
+    shape = Shape(1, 16, 32, 8, 128, "f16", 4096, kv_scale=1.0 / math.sqrt(128.0))
+    return dict(name="worked_example", seed=seed, shape=shape,
+                lens=np.array([3900, 420, 2100, 70]),
+                order=rng.permutation(shape.num_blocks).astype(np.int32))
+
+
+@dataclass
+class ContinuousSchedule:
+    """Continuous-batch schedule: fixed batch slots, Bernoulli stops, uniform replacements.
+
+    ``initial[i]`` is the prompt length of the sequence first held by slot i.
+    ``events[t]`` lists (slot, new_prompt_len) pairs: after step t the sequence in
+    that slot stops and, at step t+1, a new sequence with that prompt length takes
+    the slot.  Sequence uids are issued in order of admission: 0..n-1 for the
+    initial batch, then n, n+1, ... in (step, slot) order.
+    """
+    initial: np.ndarray
+    events: list = field(default_factory=list)
+
+
+def continuous_schedule(n: int, steps: int, seed: int, lo: int = 128, hi: int = 4096,
+                        p_stop: float = 1.0 / 200.0) -> ContinuousSchedule:
+    """Draw order: initial lengths; then per step one uniform per slot (stop if < p),
+    then one length per stopping slot in ascending slot order."""
+    rng = np.random.default_rng(seed)
+    initial = rng.integers(lo, hi + 1, size=n)
+    events = []
+    for _ in range(steps):
+        stops = np.nonzero(rng.random(n) < p_stop)[0]
+        events.append([(int(s), int(rng.integers(lo, hi + 1))) for s in stops])
+    return ContinuousSchedule(initial=initial, events=events)
+
+
+def continuous_batch(seed: int = 3, n: int = 256, steps: int = 64) -> dict:
+    """256 sequences, lengths U[128, 4096], block 16, 32 q / 8 KV heads, d128, bf16."""
+    shape = Shape(1, 16, 32, 8, 128, "bf16",
+                  num_blocks=n * ((4096 + 64 + 15) // 16), kv_scale=1.0 / math.sqrt(128.0))
+    order = np.random.default_rng(seed + 1000).permutation(shape.num_blocks).astype(np.int32)
+    return dict(name="continuous_batch", seed=seed, shape=shape, order=order,
+                schedule=continuous_schedule(n, steps, seed))
+
+
+def prefix_sharing(seed: int = 4, n: int = 64, prefix: int = 2048) -> dict:
+    """64 sequences sharing a 2048-token prefix, private suffixes U[16, 512], fp16."""
+    rng = np.random.default_rng(seed)
+    shape = Shape(1, 16, 32, 8, 128, "f16",
+                  num_blocks=prefix // 16 + n * ((512 + 16 + 15) // 16 + 1) + 64,
+                  kv_scale=1.0 / math.sqrt(128.0))
+    suffix = rng.integers(16, 512 + 1, size=n)
+    order = rng.permutation(shape.num_blocks).astype(np.int32)
+    return dict(name="prefix_sharing", seed=seed, shape=shape, prefix=prefix,
+                suffix=suffix, order=order)
+
+
+def lognormal_lengths(n: int, seed: int, median: float = 1500.0, sigma: float = 0.75,
+                      cap: int = 16384) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal(n)
+    lens = np.rint(np.exp(math.log(median) + sigma * z))
+    return np.clip(lens, 1, cap).astype(np.int64)
+
+
+def large_pool(seed: int = 5, block_size: int = 16, n: int = 384, num_layers: int = 32) -> dict:
+    """384 sequences, lognormal lengths (median 1500, sigma 0.75, cap 16384), 32 layers, fp16."""
+    lens = lognormal_lengths(n, seed)
+    # pool: every sequence's blocks after one appended token, plus two blocks of headroom each
+    nb = int(sum(-(-(int(l) + 1) // block_size) for l in lens)) + 2 * n
+    shape = Shape(num_layers, block_size, 32, 8, 128, "f16", nb, kv_scale=1.0 / math.sqrt(128.0))
+    order = np.random.default_rng(seed + 1000 * block_size).permutation(nb).astype(np.int32)
+    return dict(name=f"large_pool_b{block_size}", seed=seed, shape=shape, lens=lens, order=order)
