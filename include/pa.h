@@ -1,0 +1,215 @@
+/*
+ * pa.h -- C ABI of the paged KV-cache decode library (libpa.so, sm_100a).
+ *
+ * The problem these calls solve is stated on three pages:
+ *   [P1] "What problem does PagedAttention solve, and what is continuous batching?"
+ *   [P2] "PagedAttention & Continuous Batching"
+ *   [P3] "Continuous Batching & Paged Attention -- LLM Inference Optimization & Serving"
+ * The KV cache is stored in fixed-size physical blocks anywhere in GPU memory; a
+ * per-sequence block table maps logical block numbers to physical blocks and the
+ * attention kernel follows it when it reads keys and values ([P1] "How
+ * PagedAttention works", [P2] "Overview", [P3] "Paged attention borrows a trick
+ * from operating systems").  Decode reads the whole cache of each sequence and
+ * appends one token's keys and values per step ([P1] "Why the KV cache becomes
+ * the problem").
+ *
+ * Conventions
+ *  - Every call returns pa_status; PA_OK is 0.  A failing call leaves the host
+ *    state (free list, refcounts, tables, lengths) exactly as it was.  The text
+ *    of the last failure on the calling thread is pa_last_error().
+ *  - Device memory is owned by the caller: the key and value pools, queries,
+ *    outputs, block tables, lengths, slot mappings, copy pairs and workspaces are
+ *    raw device pointers the caller allocated.  The opaque pa_pool owns only host
+ *    metadata (free stack, refcounts, per-sequence tables and lengths).
+ *  - Device work is asynchronous on the given stream (a cudaStream_t passed as
+ *    pa_stream; NULL is the legacy default stream).  Launch failures return
+ *    PA_ERR_CUDA.  Kernels also record data errors they meet (an out-of-range
+ *    block id or slot, a length beyond the table, a bounded wait that ran out)
+ *    in a sticky device word read by pa_device_error().
+ *  - Not thread-safe: one host thread at a time per pool.
+ *
+ * Device pool layout (keys and values alike, caller-allocated, 16-byte aligned):
+ *   pool[num_layers][num_blocks][num_kv_heads][block_size][head_dim] of `dtype`.
+ * One block id names the same block in every layer, as the pages' bytes-per-token
+ * figure counts every layer ([P1] "A concrete memory example").  Slot
+ * s = block * block_size + offset names one token position inside a block.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,    /* a bad pointer, size, id, or combination */
+    PA_ERR_OUT_OF_BLOCKS = 2,  /* the free list cannot satisfy the call */
+    PA_ERR_DOUBLE_FREE = 3,    /* a block with refcount 0 was freed */
+    PA_ERR_CUDA = 4,           /* a CUDA runtime call or kernel launch failed */
+    PA_ERR_UNSUPPORTED = 5     /* a valid shape the kernels are not built for */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+typedef struct pa_pool pa_pool;
+typedef void *pa_stream;       /* a cudaStream_t */
+
+typedef struct {
+    int32_t num_layers;        /* >= 1 */
+    int32_t num_blocks;        /* physical blocks in the pool, >= 1 */
+    int32_t block_size;        /* tokens per block: 16 or 32 */
+    int32_t num_kv_heads;      /* >= 1 */
+    int32_t head_dim;          /* 64 or 128 */
+    pa_dtype dtype;            /* element type of the K and V pools */
+} pa_pool_config;
+
+typedef struct {
+    int32_t num_blocks;
+    int32_t num_free;          /* blocks on the free list */
+    int32_t num_shared;        /* blocks with refcount > 1 */
+    int32_t num_seqs;          /* live sequences */
+    int64_t num_tokens;        /* sum of live sequence lengths */
+    int64_t cow_copies;        /* copy-on-write pairs issued so far */
+    int32_t peak_used;         /* most blocks ever in use at once */
+} pa_pool_stats_t;
+
+/* Message for the last failing call on this thread ("" if none). */
+const char *pa_last_error(void);
+const char *pa_status_string(pa_status s);
+
+/* ------------------------------------------------------------------ pool */
+
+/* Create the host block manager for caller-owned device pools.
+ * [P1] "How PagedAttention works": the allocator can take any free block.  The
+ * free list is a LIFO stack; `free_order` (num_blocks ids, a permutation, may be
+ * NULL for 0..num_blocks-1) fixes which block is handed out first: free_order[0],
+ * then free_order[1], ...  k_pool / v_pool may be NULL for host-only use; the
+ * device calls then fail with PA_ERR_INVALID_ARG.  *out receives the pool. */
+pa_status pa_pool_create(const pa_pool_config *cfg, void *k_pool, void *v_pool,
+                         const int32_t *free_order, pa_pool **out);
+pa_status pa_pool_destroy(pa_pool *pool);
+pa_status pa_pool_stats(const pa_pool *pool, pa_pool_stats_t *out);
+
+/* ------------------------------------------------------------------ blocks */
+
+/* Pop the top of the free stack into *block with refcount 1.
+ * PA_ERR_OUT_OF_BLOCKS when the stack is empty ([P1] "The senior-level nuance":
+ * a full pool must queue, preempt or reject; it cannot grow). */
+pa_status pa_alloc_block(pa_pool *pool, int32_t *block);
+/* Drop one reference; at zero the block goes back on top of the stack and is
+ * reused next ([P1] "A concrete memory example": a finished request's blocks
+ * return to the pool at once).  PA_ERR_DOUBLE_FREE if the count is already 0. */
+pa_status pa_free_block(pa_pool *pool, int32_t block);
+/* Add a reference to an allocated block (sharing, [P1] "How PagedAttention
+ * works").  PA_ERR_INVALID_ARG for a free block. */
+pa_status pa_incref_block(pa_pool *pool, int32_t block);
+pa_status pa_block_refcount(const pa_pool *pool, int32_t block, int32_t *rc);
+pa_status pa_num_free_blocks(const pa_pool *pool, int32_t *n);
+/* Copy the free stack, bottom first (the last entry is handed out next), into
+ * out[0..cap); *n receives its length.  For inspection and bit-exact checks. */
+pa_status pa_free_list(const pa_pool *pool, int32_t *out, int32_t cap, int32_t *n);
+/* Host fault injection: the (n+1)-th block allocation from now fails with
+ * PA_ERR_OUT_OF_BLOCKS (n < 0 switches it off). */
+pa_status pa_debug_fail_alloc_after(pa_pool *pool, int64_t n);
+
+/* ------------------------------------------------------------------ sequences */
+
+/* New empty sequence; *seq_id receives its handle (handles are never reused). */
+pa_status pa_seq_add(pa_pool *pool, int32_t *seq_id);
+/* New sequence sharing every block of `parent` (refcount +1 each, logical order):
+ * [P1] "How PagedAttention works", beam candidates referencing the same blocks. */
+pa_status pa_seq_fork(pa_pool *pool, int32_t parent, int32_t *child);
+/* Retire a sequence: drop one reference on each of its blocks, logical order. */
+pa_status pa_seq_free(pa_pool *pool, int32_t seq_id);
+/* Length and block table of a sequence: *len tokens, *nblk blocks; the first
+ * min(cap, nblk) physical ids are written to table (table may be NULL). */
+pa_status pa_seq_info(const pa_pool *pool, int32_t seq_id, int32_t *len, int32_t *table,
+                      int32_t cap, int32_t *nblk);
+
+/* Reserve cache slots for ntok[i] new tokens of seq_ids[i], i = 0..n-1 in order,
+ * one token at a time ([P3] "Paged attention borrows a trick from operating
+ * systems": a growing request gets another block; [P1] "How PagedAttention
+ * works": a diverging sharer gets a private copy-on-write block).  For a
+ * sequence of length L:
+ *   L % block_size == 0           -> take a new block from the free stack;
+ *   else tail block refcount > 1  -> copy on write: take a new block, record the
+ *                                    pair (tail, new), drop one reference on tail,
+ *                                    and use the new block as the tail;
+ *   slot = table[L / block_size] * block_size + L % block_size;  L += 1.
+ * Outputs (host buffers): slot_mapping_out[sum(ntok)] in batch order;
+ * cow_pairs_out[2 * k] = (src, dst) for each copy, at most n pairs (one per
+ * sequence); *n_cow = k.  seq_ids must be distinct.  On PA_ERR_OUT_OF_BLOCKS
+ * nothing changes.  The caller copies the pairs to the device and calls
+ * pa_copy_blocks before writing the new tokens with pa_append_kv. */
+pa_status pa_reserve_slots(pa_pool *pool, const int32_t *seq_ids, const int32_t *ntok, int32_t n,
+                           int64_t *slot_mapping_out, int32_t *cow_pairs_out, int32_t *n_cow);
+
+/* Dense block tables for a batch (host buffers): tables_out[n][max_blocks] holds
+ * each sequence's physical ids, padded with -1; lens_out[n] its length.
+ * PA_ERR_INVALID_ARG if a sequence has more than max_blocks blocks. */
+pa_status pa_build_block_tables(const pa_pool *pool, const int32_t *seq_ids, int32_t n,
+                                int32_t max_blocks, int32_t *tables_out, int32_t *lens_out);
+
+/* ------------------------------------------------------------------ device work */
+
+/* Copy-on-write block copies: for each pair (src, dst) in pairs_dev[n_pairs][2]
+ * (device int32), block dst becomes a bit copy of block src in every layer, keys
+ * and values.  The whole block is copied, so every earlier slot stays valid. */
+pa_status pa_copy_blocks(pa_pool *pool, const int32_t *pairs_dev, int32_t n_pairs,
+                         pa_stream stream);
+
+/* Append (reshape-and-cache): row i of k_new / v_new (device, [n_tokens]
+ * [num_kv_heads][head_dim] of the pool dtype, 16-byte aligned) is bit-copied
+ * into slot slot_mapping_dev[i] of `layer`; a negative slot skips the row
+ * ([P1] "Why the KV cache becomes the problem": decode appends a small amount
+ * of new data each step). */
+pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const void *v_new,
+                       const int64_t *slot_mapping_dev, int32_t n_tokens, pa_stream stream);
+
+/* Number of splits per sequence the decode kernel uses for a table of width
+ * max_blocks when a split holds split_tokens tokens (0 = never split). */
+int32_t pa_decode_max_splits(int32_t block_size, int32_t max_blocks, int32_t split_tokens);
+/* Workspace bytes pa_decode_attention needs for that many splits (0 if 1). */
+size_t pa_decode_workspace_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t head_dim,
+                                 int32_t max_splits);
+
+/* Paged decode attention ([P1] "How PagedAttention works": the kernel follows the
+ * block table when it reads keys and values; paging does not change the result,
+ * [P1] "Common misconception").  For each sequence s and query head h, with KV
+ * head g = h / (num_q_heads / num_kv_heads) and L = seq_lens_dev[s]:
+ *   out[s][h] = sum_{j<L} softmax_j(scale * q[s][h] . K_s[j]) V_s[j],
+ *   K_s[j] = k_pool[layer][tables[s][j / B]][g][j % B], V_s likewise.
+ * q [n_seqs][num_q_heads][head_dim] in the pool dtype; out the same shape in
+ * out_dtype (PA_F32 or the pool dtype); block_tables_dev [n_seqs][max_blocks]
+ * int32, seq_lens_dev [n_seqs] int32 >= 1, all device pointers.  Sequences with
+ * more than split_tokens tokens (a multiple of block_size; 0 = never) are split
+ * into ranges of split_tokens, each reduced by a second kernel; that needs
+ * `workspace` of pa_decode_workspace_bytes(n_seqs, num_q_heads, head_dim,
+ * pa_decode_max_splits(...)) bytes (caller-owned device memory, 16-byte aligned,
+ * contents need not be initialised).  Supported: head_dim 64/128, block_size
+ * 16/32, num_q_heads / num_kv_heads in {1, 2, 4, 8}. */
+pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void *out,
+                              pa_dtype out_dtype, const int32_t *block_tables_dev,
+                              int32_t max_blocks, const int32_t *seq_lens_dev, int32_t n_seqs,
+                              int32_t num_q_heads, float scale, int32_t split_tokens,
+                              void *workspace, size_t ws_bytes, pa_stream stream);
+
+/* ------------------------------------------------------------------ diagnostics */
+
+/* Device error bits recorded by kernels since the last clear (synchronises the
+ * device): 1 = block id out of range in a table, 2 = sequence length beyond its
+ * table or < 1, 4 = a bounded wait ran out, 8 = slot out of range.  clear != 0
+ * resets the word. */
+pa_status pa_device_error(int32_t *code, int32_t clear);
+/* Kernels this library has launched since it was loaded (all devices). */
+uint64_t pa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

@@ -1,0 +1,357 @@
+// Host block manager: free stack, refcounts, per-sequence block tables,
+// slot reservation with copy-on-write.
+//
+// Follows "What problem does PagedAttention solve, and what is continuous
+// batching?", section "How PagedAttention works" (fixed-size blocks, a block
+// table per request, any free block will do, shared blocks and copy-on-write)
+// and section "A concrete memory example" (a finished request's blocks return
+// to the pool at once), and "Continuous Batching & Paged Attention", section
+// "Paged attention borrows a trick from operating systems" (a growing request
+// gets another block).  The policy choices the pages leave open -- LIFO reuse
+// over a caller-given order, logical-order reference drops, whole-call
+// rollback -- are documented in include/pa.h.
+#include <algorithm>
+#include <cstring>
+#include <new>
+
+#include "pool.hpp"
+
+namespace pa_internal {
+static thread_local std::string g_last_error;
+std::atomic<uint64_t> launch_count{0};
+
+pa_status fail(pa_status st, const std::string &msg) {
+    g_last_error = msg;
+    return st;
+}
+pa_status ok() { return PA_OK; }
+}  // namespace pa_internal
+
+using pa_internal::fail;
+
+namespace {
+
+bool valid_block(const pa_pool *p, int32_t b) { return b >= 0 && b < p->cfg.num_blocks; }
+
+void add_ref(pa_pool *p, int32_t b) {
+    if (++p->refcount[b] == 2) ++p->num_shared;
+}
+
+// Drop a reference that is known to be > 0; returns true when it reached zero.
+bool drop_ref(pa_pool *p, int32_t b) {
+    int32_t r = --p->refcount[b];
+    if (r == 1) --p->num_shared;
+    return r == 0;
+}
+
+void note_usage(pa_pool *p) {
+    int32_t used = p->cfg.num_blocks - (int32_t)p->free_stack.size();
+    p->peak_used = std::max(p->peak_used, used);
+}
+
+pa_status pop_block(pa_pool *p, int32_t *b) {
+    if (p->fail_alloc_after == 0) {
+        p->fail_alloc_after = -1;
+        return fail(PA_ERR_OUT_OF_BLOCKS, "block allocation failed (injected)");
+    }
+    if (p->free_stack.empty())
+        return fail(PA_ERR_OUT_OF_BLOCKS, "no free KV blocks left in the pool");
+    if (p->fail_alloc_after > 0) --p->fail_alloc_after;
+    *b = p->free_stack.back();
+    p->free_stack.pop_back();
+    p->refcount[*b] = 1;
+    return PA_OK;
+}
+
+// Undo journal for pa_reserve_slots: every mutation is recorded and replayed
+// backwards if the call runs out of blocks part way.
+struct Undo {
+    enum Kind { kAlloc, kDrop, kPush, kSet, kLen, kCow } kind;
+    int32_t seq;
+    int32_t a;
+    int32_t b;
+};
+
+}  // namespace
+
+extern "C" {
+
+const char *pa_last_error(void) { return pa_internal::g_last_error.c_str(); }
+
+const char *pa_status_string(pa_status s) {
+    switch (s) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_OUT_OF_BLOCKS: return "PA_ERR_OUT_OF_BLOCKS";
+    case PA_ERR_DOUBLE_FREE: return "PA_ERR_DOUBLE_FREE";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    }
+    return "PA_ERR_UNKNOWN";
+}
+
+pa_status pa_pool_create(const pa_pool_config *cfg, void *k_pool, void *v_pool,
+                         const int32_t *free_order, pa_pool **out) {
+    if (!cfg || !out) return fail(PA_ERR_INVALID_ARG, "pa_pool_create: null config or out");
+    *out = nullptr;
+    if (cfg->num_layers < 1 || cfg->num_blocks < 1 || cfg->num_kv_heads < 1 ||
+        cfg->block_size < 1 || cfg->head_dim < 1)
+        return fail(PA_ERR_INVALID_ARG, "pa_pool_create: sizes must be positive");
+    if (cfg->dtype != PA_F32 && cfg->dtype != PA_F16 && cfg->dtype != PA_BF16)
+        return fail(PA_ERR_INVALID_ARG, "pa_pool_create: unknown dtype");
+    if ((k_pool == nullptr) != (v_pool == nullptr))
+        return fail(PA_ERR_INVALID_ARG, "pa_pool_create: give both pools or neither");
+    if (((uintptr_t)k_pool | (uintptr_t)v_pool) & 15)
+        return fail(PA_ERR_INVALID_ARG, "pa_pool_create: pools must be 16-byte aligned");
+    pa_pool *p = new (std::nothrow) pa_pool();
+    if (!p) return fail(PA_ERR_INVALID_ARG, "pa_pool_create: out of host memory");
+    p->cfg = *cfg;
+    p->k_pool = k_pool;
+    p->v_pool = v_pool;
+    const int32_t nb = cfg->num_blocks;
+    p->refcount.assign(nb, 0);
+    p->free_stack.resize(nb);
+    if (free_order) {
+        std::vector<char> seen(nb, 0);
+        for (int32_t i = 0; i < nb; ++i) {
+            int32_t b = free_order[i];
+            if (b < 0 || b >= nb || seen[b]) {
+                delete p;
+                return fail(PA_ERR_INVALID_ARG, "pa_pool_create: free_order is not a permutation");
+            }
+            seen[b] = 1;
+            p->free_stack[nb - 1 - i] = b;   // free_order[0] ends on top
+        }
+    } else {
+        for (int32_t i = 0; i < nb; ++i) p->free_stack[nb - 1 - i] = i;
+    }
+    *out = p;
+    return PA_OK;
+}
+
+pa_status pa_pool_destroy(pa_pool *pool) {
+    if (!pool) return fail(PA_ERR_INVALID_ARG, "pa_pool_destroy: null pool");
+    delete pool;
+    return PA_OK;
+}
+
+pa_status pa_pool_stats(const pa_pool *p, pa_pool_stats_t *o) {
+    if (!p || !o) return fail(PA_ERR_INVALID_ARG, "pa_pool_stats: null argument");
+    o->num_blocks = p->cfg.num_blocks;
+    o->num_free = (int32_t)p->free_stack.size();
+    o->num_shared = p->num_shared;
+    o->num_seqs = (int32_t)p->seqs.size();
+    o->num_tokens = p->num_tokens;
+    o->cow_copies = p->cow_copies;
+    o->peak_used = p->peak_used;
+    return PA_OK;
+}
+
+pa_status pa_alloc_block(pa_pool *p, int32_t *block) {
+    if (!p || !block) return fail(PA_ERR_INVALID_ARG, "pa_alloc_block: null argument");
+    pa_status st = pop_block(p, block);
+    if (st == PA_OK) note_usage(p);
+    return st;
+}
+
+pa_status pa_free_block(pa_pool *p, int32_t block) {
+    if (!p || !valid_block(p, block)) return fail(PA_ERR_INVALID_ARG, "pa_free_block: bad block id");
+    if (p->refcount[block] == 0)
+        return fail(PA_ERR_DOUBLE_FREE, "pa_free_block: block " + std::to_string(block) + " is already free");
+    if (drop_ref(p, block)) p->free_stack.push_back(block);
+    return PA_OK;
+}
+
+pa_status pa_incref_block(pa_pool *p, int32_t block) {
+    if (!p || !valid_block(p, block)) return fail(PA_ERR_INVALID_ARG, "pa_incref_block: bad block id");
+    if (p->refcount[block] == 0) return fail(PA_ERR_INVALID_ARG, "pa_incref_block: block is free");
+    add_ref(p, block);
+    return PA_OK;
+}
+
+pa_status pa_block_refcount(const pa_pool *p, int32_t block, int32_t *rc) {
+    if (!p || !rc || !valid_block(p, block)) return fail(PA_ERR_INVALID_ARG, "pa_block_refcount: bad argument");
+    *rc = p->refcount[block];
+    return PA_OK;
+}
+
+pa_status pa_num_free_blocks(const pa_pool *p, int32_t *n) {
+    if (!p || !n) return fail(PA_ERR_INVALID_ARG, "pa_num_free_blocks: null argument");
+    *n = (int32_t)p->free_stack.size();
+    return PA_OK;
+}
+
+pa_status pa_free_list(const pa_pool *p, int32_t *out, int32_t cap, int32_t *n) {
+    if (!p || !n || (cap > 0 && !out)) return fail(PA_ERR_INVALID_ARG, "pa_free_list: bad argument");
+    *n = (int32_t)p->free_stack.size();
+    int32_t m = std::min<int32_t>(cap, *n);
+    if (m > 0) std::memcpy(out, p->free_stack.data(), sizeof(int32_t) * (size_t)m);
+    return PA_OK;
+}
+
+pa_status pa_debug_fail_alloc_after(pa_pool *p, int64_t n) {
+    if (!p) return fail(PA_ERR_INVALID_ARG, "pa_debug_fail_alloc_after: null pool");
+    p->fail_alloc_after = n < 0 ? -1 : n;
+    return PA_OK;
+}
+
+pa_status pa_seq_add(pa_pool *p, int32_t *seq_id) {
+    if (!p || !seq_id) return fail(PA_ERR_INVALID_ARG, "pa_seq_add: null argument");
+    if (p->next_seq == INT32_MAX) return fail(PA_ERR_INVALID_ARG, "pa_seq_add: sequence ids exhausted");
+    *seq_id = p->next_seq++;
+    p->seqs.emplace(*seq_id, pa_pool::Seq());
+    return PA_OK;
+}
+
+pa_status pa_seq_fork(pa_pool *p, int32_t parent, int32_t *child) {
+    if (!p || !child) return fail(PA_ERR_INVALID_ARG, "pa_seq_fork: null argument");
+    auto it = p->seqs.find(parent);
+    if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_seq_fork: unknown parent");
+    if (p->next_seq == INT32_MAX) return fail(PA_ERR_INVALID_ARG, "pa_seq_fork: sequence ids exhausted");
+    pa_pool::Seq s = it->second;          // copy of table and length
+    for (int32_t b : s.table) add_ref(p, b);
+    *child = p->next_seq++;
+    p->num_tokens += s.len;
+    p->seqs.emplace(*child, std::move(s));
+    return PA_OK;
+}
+
+pa_status pa_seq_free(pa_pool *p, int32_t seq_id) {
+    if (!p) return fail(PA_ERR_INVALID_ARG, "pa_seq_free: null pool");
+    auto it = p->seqs.find(seq_id);
+    if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_seq_free: unknown sequence");
+    for (int32_t b : it->second.table)
+        if (drop_ref(p, b)) p->free_stack.push_back(b);
+    p->num_tokens -= it->second.len;
+    p->seqs.erase(it);
+    return PA_OK;
+}
+
+pa_status pa_seq_info(const pa_pool *p, int32_t seq_id, int32_t *len, int32_t *table, int32_t cap,
+                      int32_t *nblk) {
+    if (!p) return fail(PA_ERR_INVALID_ARG, "pa_seq_info: null pool");
+    auto it = p->seqs.find(seq_id);
+    if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_seq_info: unknown sequence");
+    const pa_pool::Seq &s = it->second;
+    if (len) *len = s.len;
+    if (nblk) *nblk = (int32_t)s.table.size();
+    if (table && cap > 0) {
+        int32_t m = std::min<int32_t>(cap, (int32_t)s.table.size());
+        std::memcpy(table, s.table.data(), sizeof(int32_t) * (size_t)m);
+    }
+    return PA_OK;
+}
+
+pa_status pa_reserve_slots(pa_pool *p, const int32_t *seq_ids, const int32_t *ntok, int32_t n,
+                           int64_t *slot_mapping_out, int32_t *cow_pairs_out, int32_t *n_cow) {
+    if (!p || n < 0 || (n > 0 && (!seq_ids || !ntok)))
+        return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: bad argument");
+    int64_t total = 0;
+    std::vector<pa_pool::Seq *> seqs((size_t)n);
+    for (int32_t i = 0; i < n; ++i) {
+        auto it = p->seqs.find(seq_ids[i]);
+        if (it == p->seqs.end() || ntok[i] < 0)
+            return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: unknown sequence or negative count");
+        if ((int64_t)it->second.len + ntok[i] > INT32_MAX)
+            return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: sequence too long");
+        seqs[i] = &it->second;
+        total += ntok[i];
+    }
+    {   // distinct ids
+        std::vector<int32_t> ids(seq_ids, seq_ids + n);
+        std::sort(ids.begin(), ids.end());
+        if (std::adjacent_find(ids.begin(), ids.end()) != ids.end())
+            return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: duplicate sequence id");
+    }
+    if (total > 0 && !slot_mapping_out) return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: null slot_mapping_out");
+
+    const int32_t B = p->cfg.block_size;
+    std::vector<Undo> journal;
+    int32_t cows = 0;
+    int64_t k = 0;
+    pa_status st = PA_OK;
+    for (int32_t i = 0; i < n && st == PA_OK; ++i) {
+        pa_pool::Seq &s = *seqs[i];
+        for (int32_t t = 0; t < ntok[i]; ++t) {
+            const int32_t L = s.len;
+            if (L % B == 0) {
+                int32_t b;
+                st = pop_block(p, &b);
+                if (st != PA_OK) break;
+                journal.push_back({Undo::kAlloc, seq_ids[i], b, 0});
+                s.table.push_back(b);
+                journal.push_back({Undo::kPush, seq_ids[i], 0, 0});
+            } else {
+                const int32_t tail = s.table.back();
+                if (p->refcount[tail] > 1) {
+                    int32_t nb;
+                    st = pop_block(p, &nb);
+                    if (st != PA_OK) break;
+                    journal.push_back({Undo::kAlloc, seq_ids[i], nb, 0});
+                    drop_ref(p, tail);
+                    journal.push_back({Undo::kDrop, seq_ids[i], tail, 0});
+                    const int32_t idx = (int32_t)s.table.size() - 1;
+                    s.table[idx] = nb;
+                    journal.push_back({Undo::kSet, seq_ids[i], idx, tail});
+                    if (cow_pairs_out) {
+                        cow_pairs_out[2 * cows] = tail;
+                        cow_pairs_out[2 * cows + 1] = nb;
+                    }
+                    ++cows;
+                    journal.push_back({Undo::kCow, seq_ids[i], 0, 0});
+                }
+            }
+            slot_mapping_out[k++] = (int64_t)s.table[L / B] * B + L % B;
+            s.len = L + 1;
+            journal.push_back({Undo::kLen, seq_ids[i], L, 0});
+        }
+    }
+    if (st != PA_OK) {
+        std::string msg = pa_last_error();
+        for (auto it = journal.rbegin(); it != journal.rend(); ++it) {
+            pa_pool::Seq &s = p->seqs[it->seq];
+            switch (it->kind) {
+            case Undo::kAlloc:
+                p->refcount[it->a] = 0;
+                p->free_stack.push_back(it->a);
+                break;
+            case Undo::kDrop: add_ref(p, it->a); break;
+            case Undo::kPush: s.table.pop_back(); break;
+            case Undo::kSet: s.table[it->a] = it->b; break;
+            case Undo::kLen: s.len = it->a; break;
+            case Undo::kCow: break;
+            }
+        }
+        return fail(st, "pa_reserve_slots: " + msg + " (no change made)");
+    }
+    p->num_tokens += total;
+    p->cow_copies += cows;
+    if (n_cow) *n_cow = cows;
+    note_usage(p);
+    return PA_OK;
+}
+
+pa_status pa_build_block_tables(const pa_pool *p, const int32_t *seq_ids, int32_t n, int32_t max_blocks,
+                                int32_t *tables_out, int32_t *lens_out) {
+    if (!p || n < 0 || max_blocks < 1 || (n > 0 && (!seq_ids || !tables_out || !lens_out)))
+        return fail(PA_ERR_INVALID_ARG, "pa_build_block_tables: bad argument");
+    for (int32_t i = 0; i < n; ++i) {
+        auto it = p->seqs.find(seq_ids[i]);
+        if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_build_block_tables: unknown sequence");
+        if ((int32_t)it->second.table.size() > max_blocks)
+            return fail(PA_ERR_INVALID_ARG, "pa_build_block_tables: sequence has more than max_blocks blocks");
+    }
+    for (int32_t i = 0; i < n; ++i) {
+        const pa_pool::Seq &s = p->seqs.find(seq_ids[i])->second;
+        int32_t *row = tables_out + (size_t)i * max_blocks;
+        const size_t nb = s.table.size();
+        if (nb) std::memcpy(row, s.table.data(), sizeof(int32_t) * nb);
+        std::fill(row + nb, row + max_blocks, -1);
+        lens_out[i] = s.len;
+    }
+    return PA_OK;
+}
+
+uint64_t pa_launch_count(void) { return pa_internal::launch_count.load(); }
+
+}  // extern "C"

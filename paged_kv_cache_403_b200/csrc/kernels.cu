@@ -1,0 +1,756 @@
+// sm_100a kernels of the paged decode path and their C ABI entry points.
+//
+//  paged_decode_kernel  -- single-query decode attention through the block
+//                          table ("What problem does PagedAttention solve, and
+//                          what is continuous batching?", "How PagedAttention
+//                          works": the kernel follows the table when it reads
+//                          keys and values).  One CTA per (sequence, group of up
+//                          to 4 query heads sharing one KV head, split).
+//  split_reduce_kernel  -- log-sum-exp merge of the splits of long sequences.
+//  append_kv_kernel     -- reshape-and-cache: new K/V rows into their slots
+//                          (same page, "Why the KV cache becomes the problem":
+//                          decode appends a small amount of new data).
+//  copy_blocks_kernel   -- copy-on-write block copies (same page, "How
+//                          PagedAttention works").
+//
+// Design (B200): each (block, KV head) tile of keys or values is one contiguous
+// block_size x head_dim run in HBM, fetched whole by a 1-D TMA bulk copy
+// (cp.async.bulk, no tensor map, no multicast) into a ring of shared-memory
+// stages guarded by mbarriers.  A producer warp walks the block table and keeps
+// the ring full; four consumer warps each own whole tiles.  Inside a warp eight
+// lanes share one token (16-byte vector reads of the row), so a pass covers four
+// tokens; dot products reduce over the eight lanes with xor shuffles.  Every
+// query head of the GQA group reuses the same key/value registers, so K and V
+// are read from HBM once per KV head.  The softmax is online in base 2 (q is
+// pre-scaled by scale*log2(e)); the running maximum is only moved when a score
+// exceeds it by more than 2^8, which keeps rescaling off the common path and is
+// exact because the final division uses the same reference maximum.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <string>
+
+#include "pool.hpp"
+
+using pa_internal::fail;
+
+namespace {
+
+// ------------------------------------------------------------------ device error word
+constexpr unsigned kErrBadBlock = 1u, kErrBadLen = 2u, kErrTimeout = 4u, kErrBadSlot = 8u;
+__device__ unsigned int g_device_error = 0;
+
+__device__ __forceinline__ void raise_error(unsigned e) { atomicOr(&g_device_error, e); }
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Waits are bounded: after kWaitLimitNs the waiter records kErrTimeout and gives up.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// One thread waits (the producer lane).
+__device__ __forceinline__ bool mbar_wait_thread(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            raise_error(kErrTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// A whole warp waits and leaves together, so later full-warp shuffles stay converged.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        const bool done = mbar_try_wait(bar, parity);
+        if (__all_sync(0xffffffffu, done)) return true;
+        if (it == 0) t0 = global_timer_ns();
+        const bool late = global_timer_ns() - t0 > kWaitLimitNs;
+        if (__any_sync(0xffffffffu, late)) {
+            if ((threadIdx.x & 31) == 0) raise_error(kErrTimeout);
+            return false;
+        }
+    }
+}
+
+// 1-D TMA bulk copy global -> shared, completing `bytes` transactions on `bar`.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// ------------------------------------------------------------------ element types
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<float> {
+    static constexpr int kVec = 4;   // elements per 16 bytes
+    __device__ __forceinline__ static void widen(const uint4 &u, float *f) {
+        f[0] = __uint_as_float(u.x);
+        f[1] = __uint_as_float(u.y);
+        f[2] = __uint_as_float(u.z);
+        f[3] = __uint_as_float(u.w);
+    }
+    __device__ __forceinline__ static float narrow(float x) { return x; }
+};
+
+template <>
+struct Elem<__half> {
+    static constexpr int kVec = 8;
+    __device__ __forceinline__ static void widen2(uint32_t w, float *f) {
+        __half2 h;
+        memcpy(&h, &w, 4);
+        const float2 x = __half22float2(h);
+        f[0] = x.x;
+        f[1] = x.y;
+    }
+    __device__ __forceinline__ static void widen(const uint4 &u, float *f) {
+        widen2(u.x, f);
+        widen2(u.y, f + 2);
+        widen2(u.z, f + 4);
+        widen2(u.w, f + 6);
+    }
+    __device__ __forceinline__ static __half narrow(float x) { return __float2half_rn(x); }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+    static constexpr int kVec = 8;
+    // bf16 is the top half of an fp32: the low element of a word is (w << 16),
+    // the high one (w & 0xffff0000).
+    __device__ __forceinline__ static void widen2(uint32_t w, float *f) {
+        f[0] = __uint_as_float(w << 16);
+        f[1] = __uint_as_float(w & 0xffff0000u);
+    }
+    __device__ __forceinline__ static void widen(const uint4 &u, float *f) {
+        widen2(u.x, f);
+        widen2(u.y, f + 2);
+        widen2(u.z, f + 4);
+        widen2(u.w, f + 6);
+    }
+    __device__ __forceinline__ static __nv_bfloat16 narrow(float x) { return __float2bfloat16_rn(x); }
+};
+
+// ------------------------------------------------------------------ decode attention
+constexpr int kLanesPerToken = 8;                        // lanes sharing one token row
+constexpr int kTokensPerPass = 32 / kLanesPerToken;      // tokens a warp covers per pass
+constexpr int kConsumerWarps = 4;
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+constexpr float kRescaleThreshold = 8.0f;                // log2 units: 2^8 headroom
+
+struct DecodeParams {
+    const unsigned char *k_layer;   // this layer's key pool [NB][Hkv][B][D]
+    const unsigned char *v_layer;
+    const void *q;                  // [n][Hq][D]
+    void *out;                      // [n][Hq][D]
+    const int32_t *tables;          // [n][max_blocks]
+    const int32_t *lens;            // [n]
+    float *ws_acc;                  // [n][max_splits][Hq][D]
+    float *ws_ml;                   // [n][max_splits][Hq][2]
+    int32_t n_seqs, max_blocks, num_blocks, num_kv_heads, num_q_heads;
+    int32_t split_blocks, max_splits, out_f32;
+    float scale_log2;
+};
+
+template <typename T, int B, int D>
+struct DecodeShape {
+    static constexpr int kVec = Elem<T>::kVec;
+    static constexpr int kElems = D / kLanesPerToken;      // elements of a row per lane
+    static constexpr int kChunks = kElems / kVec;          // 16-byte chunks per lane
+    static constexpr int kRowBytes = D * (int)sizeof(T);
+    static constexpr int kTileBytes = B * kRowBytes;
+    static constexpr int kStages = (2 * kTileBytes <= 8192) ? 8 : 4;
+    static_assert(kChunks >= 1 && kElems % kVec == 0, "row must split into 16-byte chunks");
+    static_assert(kStages % kConsumerWarps == 0, "each stage must belong to one consumer warp");
+    static constexpr int kRingBytes = kStages * 2 * kTileBytes;
+};
+
+template <int HPC, int D>
+constexpr int reduce_bytes() {
+    return kConsumerWarps * HPC * (2 + D) * 4;
+}
+
+template <typename T, int B, int D, int HPC>
+constexpr size_t decode_smem_bytes() {
+    using S = DecodeShape<T, B, D>;
+    return (size_t)S::kRingBytes + 2 * S::kStages * sizeof(uint64_t) + reduce_bytes<HPC, D>();
+}
+
+template <typename T>
+__device__ __forceinline__ void store_out(const DecodeParams &p, size_t idx, float v) {
+    if (p.out_f32)
+        static_cast<float *>(p.out)[idx] = v;
+    else
+        static_cast<T *>(p.out)[idx] = Elem<T>::narrow(v);
+}
+
+template <typename T, int B, int D, int HPC>
+__global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const DecodeParams p) {
+    using EL = Elem<T>;
+    using SH = DecodeShape<T, B, D>;
+    constexpr int VEC = SH::kVec, E = SH::kElems, NCH = SH::kChunks, ROW = SH::kRowBytes;
+    constexpr int TILE = SH::kTileBytes, STAGES = SH::kStages;
+    extern __shared__ __align__(128) unsigned char smem[];
+
+    const int s = blockIdx.x;
+    const int hg = blockIdx.y;
+    const int split = blockIdx.z;
+
+    int L = p.lens[s];
+    if (L < 1 || (L + B - 1) / B > p.max_blocks) {
+        if (threadIdx.x == 0 && hg == 0 && split == 0) raise_error(kErrBadLen);
+        if (L < 1) {   // nothing to attend to: defined output 0
+            if (split == 0)
+                for (int t = threadIdx.x; t < HPC * D; t += blockDim.x)
+                    store_out<T>(p, ((size_t)s * p.num_q_heads + hg * HPC + t / D) * D + t % D, 0.f);
+            return;
+        }
+        L = p.max_blocks * B;
+    }
+    const int nblk = (L + B - 1) / B;
+    const int b0 = split * p.split_blocks;
+    if (b0 >= nblk) return;
+    const int b1 = min(nblk, b0 + p.split_blocks);
+    const int ntiles = b1 - b0;
+    const int nsplit = (nblk + p.split_blocks - 1) / p.split_blocks;
+    const int group = p.num_q_heads / p.num_kv_heads;
+    const int h0 = hg * HPC;
+    const int g = h0 / group;
+
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + SH::kRingBytes);
+    uint64_t *empty = full + STAGES;
+    float *red_m = reinterpret_cast<float *>(empty + STAGES);   // [warps][HPC]
+    float *red_l = red_m + kConsumerWarps * HPC;                 // [warps][HPC]
+    float *red_o = red_l + kConsumerWarps * HPC;                 // [warps][HPC][D]
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_fence_init();
+    }
+    __syncthreads();
+
+    if (warp == kConsumerWarps) {
+        // ---------------- producer: walk the table, keep the ring full
+        const int32_t *trow = p.tables + (size_t)s * p.max_blocks + b0;
+        bool ok = true;
+        for (int base = 0; base < ntiles && ok; base += 32) {
+            int blk = 0;
+            if (base + lane < ntiles) {
+                blk = trow[base + lane];
+                if ((unsigned)blk >= (unsigned)p.num_blocks) {
+                    raise_error(kErrBadBlock);
+                    blk = 0;   // stay in bounds; the error word reports the bad table
+                }
+            }
+            const int cnt = min(32, ntiles - base);
+            for (int j = 0; j < cnt; ++j) {
+                const int b = __shfl_sync(0xffffffffu, blk, j);
+                const int i = base + j;
+                const int st = i % STAGES;
+                if (lane == 0) {
+                    if (i >= STAGES) ok = mbar_wait_thread(&empty[st], ((i / STAGES) - 1) & 1);
+                    if (ok) {
+                        const size_t off = ((size_t)b * p.num_kv_heads + g) * TILE;
+                        unsigned char *dst = smem + st * 2 * TILE;
+                        mbar_arrive_expect_tx(&full[st], 2 * TILE);
+                        bulk_g2s(dst, p.k_layer + off, TILE, &full[st]);
+                        bulk_g2s(dst + TILE, p.v_layer + off, TILE, &full[st]);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+            }
+        }
+    } else {
+        // ---------------- consumers
+        const int c = lane % kLanesPerToken;       // which 16-byte chunks of the row
+        const int slot = lane / kLanesPerToken;    // which token of the pass
+        float q[HPC][E];
+#pragma unroll
+        for (int h = 0; h < HPC; ++h) {
+            const T *qrow = static_cast<const T *>(p.q) + ((size_t)s * p.num_q_heads + h0 + h) * D;
+#pragma unroll
+            for (int k = 0; k < NCH; ++k) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(qrow + (k * kLanesPerToken + c) * VEC);
+                float f[VEC];
+                EL::widen(u, f);
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) q[h][k * VEC + v] = f[v] * p.scale_log2;
+            }
+        }
+        float m[HPC], l[HPC], o[HPC][E];
+#pragma unroll
+        for (int h = 0; h < HPC; ++h) {
+            m[h] = -INFINITY;
+            l[h] = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) o[h][e] = 0.f;
+        }
+
+        for (int i = warp; i < ntiles; i += kConsumerWarps) {
+            const int st = i % STAGES;
+            if (!mbar_wait_warp(&full[st], (i / STAGES) & 1)) break;
+            const unsigned char *kt = smem + st * 2 * TILE;
+            const unsigned char *vt = kt + TILE;
+            const int tok0 = (b0 + i) * B;
+#pragma unroll 2
+            for (int ps = 0; ps < B / kTokensPerPass; ++ps) {
+                const int r = ps * kTokensPerPass + slot;
+                const bool valid = tok0 + r < L;
+                float kf[E];
+#pragma unroll
+                for (int k = 0; k < NCH; ++k) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(kt + r * ROW + (k * kLanesPerToken + c) * 16);
+                    EL::widen(u, &kf[k * VEC]);
+                }
+                float sc[HPC];
+#pragma unroll
+                for (int h = 0; h < HPC; ++h) {
+                    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                    for (int e = 0; e < E; e += 2) {
+                        a0 = fmaf(q[h][e], kf[e], a0);
+                        a1 = fmaf(q[h][e + 1], kf[e + 1], a1);
+                    }
+                    sc[h] = a0 + a1;
+                }
+#pragma unroll
+                for (int off = 1; off < kLanesPerToken; off <<= 1)
+#pragma unroll
+                    for (int h = 0; h < HPC; ++h) sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], off);
+                float pr[HPC];
+#pragma unroll
+                for (int h = 0; h < HPC; ++h) {
+                    const float sv = valid ? sc[h] : -INFINITY;
+                    if (sv > m[h] + kRescaleThreshold) {
+                        const float f = ex2(m[h] - sv);
+                        l[h] *= f;
+#pragma unroll
+                        for (int e = 0; e < E; ++e) o[h][e] *= f;
+                        m[h] = sv;
+                    }
+                    pr[h] = valid ? ex2(sv - m[h]) : 0.f;
+                    l[h] += pr[h];
+                }
+                if (valid) {
+                    float vf[E];
+#pragma unroll
+                    for (int k = 0; k < NCH; ++k) {
+                        const uint4 u =
+                            *reinterpret_cast<const uint4 *>(vt + r * ROW + (k * kLanesPerToken + c) * 16);
+                        EL::widen(u, &vf[k * VEC]);
+                    }
+#pragma unroll
+                    for (int h = 0; h < HPC; ++h)
+#pragma unroll
+                        for (int e = 0; e < E; ++e) o[h][e] = fmaf(pr[h], vf[e], o[h][e]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+
+        // merge the four token slots of the warp (lanes differing in bits 3 and 4)
+#pragma unroll
+        for (int off = kLanesPerToken; off < 32; off <<= 1) {
+#pragma unroll
+            for (int h = 0; h < HPC; ++h) {
+                const float mo = __shfl_xor_sync(0xffffffffu, m[h], off);
+                const float lo = __shfl_xor_sync(0xffffffffu, l[h], off);
+                const float mn = fmaxf(m[h], mo);
+                const float fa = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - mn);
+                const float fb = (mo == -INFINITY) ? 0.f : ex2(mo - mn);
+                l[h] = l[h] * fa + lo * fb;
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const float oo = __shfl_xor_sync(0xffffffffu, o[h][e], off);
+                    o[h][e] = o[h][e] * fa + oo * fb;
+                }
+                m[h] = mn;
+            }
+        }
+        if (lane < kLanesPerToken) {
+#pragma unroll
+            for (int h = 0; h < HPC; ++h) {
+                if (lane == 0) {
+                    red_m[warp * HPC + h] = m[h];
+                    red_l[warp * HPC + h] = l[h];
+                }
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int d = ((e / VEC) * kLanesPerToken + c) * VEC + e % VEC;
+                    red_o[(warp * HPC + h) * D + d] = o[h][e];
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // merge the consumer warps and write the result or this split's partial
+    for (int t = threadIdx.x; t < HPC * D; t += blockDim.x) {
+        const int h = t / D;
+        const int d = t % D;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, red_m[w * HPC + h]);
+        float lsum = 0.f, osum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+            const float mw = red_m[w * HPC + h];
+            const float f = (mw == -INFINITY) ? 0.f : ex2(mw - mx);
+            lsum += red_l[w * HPC + h] * f;
+            osum += red_o[(w * HPC + h) * D + d] * f;
+        }
+        const int hq = h0 + h;
+        if (nsplit == 1) {
+            store_out<T>(p, ((size_t)s * p.num_q_heads + hq) * D + d, osum / lsum);
+        } else {
+            const size_t part = ((size_t)s * p.max_splits + split) * p.num_q_heads + hq;
+            p.ws_acc[part * D + d] = osum;
+            if (d == 0) {
+                p.ws_ml[part * 2] = mx;
+                p.ws_ml[part * 2 + 1] = lsum;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ split reduce
+template <typename T, int B, int D>
+__global__ void __launch_bounds__(D) split_reduce_kernel(const DecodeParams p) {
+    const int s = blockIdx.x;
+    const int hq = blockIdx.y;
+    const int d = threadIdx.x;
+    int L = p.lens[s];
+    if (L < 1) return;
+    if ((L + B - 1) / B > p.max_blocks) L = p.max_blocks * B;
+    const int nblk = (L + B - 1) / B;
+    const int nsplit = (nblk + p.split_blocks - 1) / p.split_blocks;
+    if (nsplit <= 1) return;
+    const size_t base = (size_t)s * p.max_splits * p.num_q_heads + hq;
+    float mx = -INFINITY;
+    for (int x = 0; x < nsplit; ++x) mx = fmaxf(mx, p.ws_ml[(base + (size_t)x * p.num_q_heads) * 2]);
+    float lsum = 0.f, osum = 0.f;
+    for (int x = 0; x < nsplit; ++x) {
+        const size_t part = base + (size_t)x * p.num_q_heads;
+        const float f = ex2(p.ws_ml[part * 2] - mx);
+        lsum += p.ws_ml[part * 2 + 1] * f;
+        osum += p.ws_acc[part * D + d] * f;
+    }
+    store_out<T>(p, ((size_t)s * p.num_q_heads + hq) * D + d, osum / lsum);
+}
+
+// ------------------------------------------------------------------ append / copy
+struct AppendParams {
+    unsigned char *k_layer;
+    unsigned char *v_layer;
+    const unsigned char *k_new;     // [n][Hkv][D]
+    const unsigned char *v_new;
+    const int64_t *slots;
+    int32_t n_tokens, block_size, num_kv_heads, row_chunks;   // row_chunks = D*e/16
+    int64_t num_blocks;
+};
+
+__global__ void __launch_bounds__(128) append_kv_kernel(const AppendParams p) {
+    const int chunks = p.num_kv_heads * p.row_chunks;   // 16-byte chunks per token
+    for (int i = blockIdx.x; i < p.n_tokens; i += gridDim.x) {
+        const int64_t slot = p.slots[i];
+        if (slot < 0) continue;
+        const int64_t blk = slot / p.block_size;
+        const int off = (int)(slot % p.block_size);
+        if (blk >= p.num_blocks) {
+            if (threadIdx.x == 0) raise_error(kErrBadSlot);
+            continue;
+        }
+        for (int t = threadIdx.x; t < chunks; t += blockDim.x) {
+            const int h = t / p.row_chunks;
+            const int c = t % p.row_chunks;
+            const size_t dst = (((size_t)blk * p.num_kv_heads + h) * p.block_size + off) * p.row_chunks + c;
+            const size_t src = ((size_t)i * p.num_kv_heads + h) * p.row_chunks + c;
+            reinterpret_cast<uint4 *>(p.k_layer)[dst] = reinterpret_cast<const uint4 *>(p.k_new)[src];
+            reinterpret_cast<uint4 *>(p.v_layer)[dst] = reinterpret_cast<const uint4 *>(p.v_new)[src];
+        }
+    }
+}
+
+struct CopyParams {
+    unsigned char *k_pool;
+    unsigned char *v_pool;
+    const int32_t *pairs;     // [n][2] (src, dst)
+    int64_t block_chunks;     // 16-byte chunks per block (all heads)
+    int64_t layer_chunks;     // 16-byte chunks per layer
+    int32_t num_blocks;
+};
+
+__global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p) {
+    const int pair = blockIdx.x;
+    const int layer = blockIdx.y;
+    const int src = p.pairs[2 * pair];
+    const int dst = p.pairs[2 * pair + 1];
+    if ((unsigned)src >= (unsigned)p.num_blocks || (unsigned)dst >= (unsigned)p.num_blocks) {
+        if (threadIdx.x == 0) raise_error(kErrBadBlock);
+        return;
+    }
+    uint4 *pool = reinterpret_cast<uint4 *>(blockIdx.z == 0 ? p.k_pool : p.v_pool);
+    uint4 *from = pool + layer * p.layer_chunks + (int64_t)src * p.block_chunks;
+    uint4 *to = pool + layer * p.layer_chunks + (int64_t)dst * p.block_chunks;
+    for (int64_t t = threadIdx.x; t < p.block_chunks; t += blockDim.x) to[t] = from[t];
+}
+
+// ------------------------------------------------------------------ host dispatch
+pa_status check_launch(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+    return PA_OK;
+}
+
+// Raise the dynamic shared-memory limit of one kernel once per device; `done` is
+// the caller's per-kernel flag array (one per template instantiation).
+template <typename K>
+pa_status ensure_smem(K kernel, size_t bytes, bool (&done)[64]) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return fail(PA_ERR_CUDA, "cudaGetDevice failed");
+    if (dev < 64 && done[dev]) return PA_OK;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+    if (dev < 64) done[dev] = true;
+    return PA_OK;
+}
+
+template <typename T, int B, int D, int HPC>
+pa_status launch_decode(const DecodeParams &p, cudaStream_t stream) {
+    constexpr size_t smem = decode_smem_bytes<T, B, D, HPC>();
+    auto kernel = paged_decode_kernel<T, B, D, HPC>;
+    static bool smem_set[64] = {};
+    pa_status st = ensure_smem(kernel, smem, smem_set);
+    if (st != PA_OK) return st;
+    dim3 grid(p.n_seqs, p.num_q_heads / HPC, p.max_splits);
+    kernel<<<grid, kDecodeThreads, smem, stream>>>(p);
+    pa_internal::launch_count.fetch_add(1);
+    st = check_launch("paged_decode_kernel");
+    if (st != PA_OK || p.max_splits <= 1) return st;
+    split_reduce_kernel<T, B, D><<<dim3(p.n_seqs, p.num_q_heads), D, 0, stream>>>(p);
+    pa_internal::launch_count.fetch_add(1);
+    return check_launch("split_reduce_kernel");
+}
+
+template <typename T, int B, int D>
+pa_status dispatch_hpc(const DecodeParams &p, int hpc, cudaStream_t stream) {
+    switch (hpc) {
+    case 1: return launch_decode<T, B, D, 1>(p, stream);
+    case 2: return launch_decode<T, B, D, 2>(p, stream);
+    case 4: return launch_decode<T, B, D, 4>(p, stream);
+    }
+    return fail(PA_ERR_UNSUPPORTED, "unsupported query heads per KV head");
+}
+
+template <typename T>
+pa_status dispatch_shape(const DecodeParams &p, int B, int D, int hpc, cudaStream_t stream) {
+    if (B == 16 && D == 128) return dispatch_hpc<T, 16, 128>(p, hpc, stream);
+    if (B == 32 && D == 128) return dispatch_hpc<T, 32, 128>(p, hpc, stream);
+    if (B == 16 && D == 64) return dispatch_hpc<T, 16, 64>(p, hpc, stream);
+    if (B == 32 && D == 64) return dispatch_hpc<T, 32, 64>(p, hpc, stream);
+    return fail(PA_ERR_UNSUPPORTED, "block_size must be 16 or 32 and head_dim 64 or 128");
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t pa_decode_max_splits(int32_t block_size, int32_t max_blocks, int32_t split_tokens) {
+    if (block_size < 1 || max_blocks < 1 || split_tokens < 0) return 0;
+    if (split_tokens == 0) return 1;
+    const int32_t split_blocks = split_tokens / block_size;
+    if (split_blocks < 1) return 0;
+    return (max_blocks + split_blocks - 1) / split_blocks;
+}
+
+size_t pa_decode_workspace_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_splits) {
+    if (n_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_splits <= 1) return 0;
+    const size_t parts = (size_t)n_seqs * max_splits * num_q_heads;
+    return parts * head_dim * sizeof(float) + parts * 2 * sizeof(float);
+}
+
+pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void *out, pa_dtype out_dtype,
+                              const int32_t *block_tables_dev, int32_t max_blocks, const int32_t *seq_lens_dev,
+                              int32_t n_seqs, int32_t num_q_heads, float scale, int32_t split_tokens,
+                              void *workspace, size_t ws_bytes, pa_stream stream) {
+    if (!pool || !pool->k_pool) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: pool has no device memory");
+    const pa_pool_config &c = pool->cfg;
+    if (layer < 0 || layer >= c.num_layers) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: layer out of range");
+    if (n_seqs < 0 || max_blocks < 1) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: bad n_seqs/max_blocks");
+    if (n_seqs == 0) return PA_OK;
+    if (!q || !out || !block_tables_dev || !seq_lens_dev)
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: null device pointer");
+    if (!aligned16(q) || !aligned16(out) || ((uintptr_t)block_tables_dev & 3) || ((uintptr_t)seq_lens_dev & 3))
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: misaligned pointer");
+    if (out_dtype != PA_F32 && out_dtype != c.dtype)
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: out_dtype must be PA_F32 or the pool dtype");
+    if (num_q_heads < 1 || num_q_heads % c.num_kv_heads != 0)
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: num_q_heads must be a multiple of num_kv_heads");
+    const int group = num_q_heads / c.num_kv_heads;
+    if (group != 1 && group != 2 && group != 4 && group != 8)
+        return fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: query heads per KV head must be 1, 2, 4 or 8");
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: scale must be finite");
+    if (split_tokens < 0 || (split_tokens > 0 && split_tokens % c.block_size != 0))
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: split_tokens must be 0 or a multiple of block_size");
+    const int32_t max_splits = pa_decode_max_splits(c.block_size, max_blocks, split_tokens);
+    const int hpc = group < 4 ? group : 4;
+    if (max_splits > 65535 || num_q_heads / hpc > 65535)
+        return fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: grid too large");
+    const size_t need = pa_decode_workspace_bytes(n_seqs, num_q_heads, c.head_dim, max_splits);
+    if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: workspace missing, misaligned or smaller than " +
+                                            std::to_string(need) + " bytes");
+
+    DecodeParams p;
+    p.k_layer = static_cast<const unsigned char *>(pool->k_pool) + (size_t)layer * pool->layer_bytes();
+    p.v_layer = static_cast<const unsigned char *>(pool->v_pool) + (size_t)layer * pool->layer_bytes();
+    p.q = q;
+    p.out = out;
+    p.tables = block_tables_dev;
+    p.lens = seq_lens_dev;
+    const size_t parts = (size_t)n_seqs * max_splits * num_q_heads;
+    p.ws_acc = static_cast<float *>(workspace);
+    p.ws_ml = need > 0 ? static_cast<float *>(workspace) + parts * c.head_dim : nullptr;
+    p.n_seqs = n_seqs;
+    p.max_blocks = max_blocks;
+    p.num_blocks = c.num_blocks;
+    p.num_kv_heads = c.num_kv_heads;
+    p.num_q_heads = num_q_heads;
+    p.split_blocks = split_tokens > 0 ? split_tokens / c.block_size : max_blocks;
+    p.max_splits = max_splits;
+    p.out_f32 = out_dtype == PA_F32;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);   // scale * log2(e)
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (c.dtype) {
+    case PA_F32: return dispatch_shape<float>(p, c.block_size, c.head_dim, hpc, st);
+    case PA_F16: return dispatch_shape<__half>(p, c.block_size, c.head_dim, hpc, st);
+    case PA_BF16: return dispatch_shape<__nv_bfloat16>(p, c.block_size, c.head_dim, hpc, st);
+    }
+    return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: unknown dtype");
+}
+
+pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const void *v_new,
+                       const int64_t *slot_mapping_dev, int32_t n_tokens, pa_stream stream) {
+    if (!pool || !pool->k_pool) return fail(PA_ERR_INVALID_ARG, "pa_append_kv: pool has no device memory");
+    if (layer < 0 || layer >= pool->cfg.num_layers) return fail(PA_ERR_INVALID_ARG, "pa_append_kv: layer out of range");
+    if (n_tokens < 0) return fail(PA_ERR_INVALID_ARG, "pa_append_kv: negative n_tokens");
+    if (n_tokens == 0) return PA_OK;
+    if (!k_new || !v_new || !slot_mapping_dev || !aligned16(k_new) || !aligned16(v_new) ||
+        ((uintptr_t)slot_mapping_dev & 7))
+        return fail(PA_ERR_INVALID_ARG, "pa_append_kv: null or misaligned device pointer");
+    const size_t row_bytes = (size_t)pool->cfg.head_dim * pool->elem_bytes();
+    if (row_bytes % 16) return fail(PA_ERR_UNSUPPORTED, "pa_append_kv: head_dim * element size must be a multiple of 16");
+    AppendParams p;
+    p.k_layer = static_cast<unsigned char *>(pool->k_pool) + (size_t)layer * pool->layer_bytes();
+    p.v_layer = static_cast<unsigned char *>(pool->v_pool) + (size_t)layer * pool->layer_bytes();
+    p.k_new = static_cast<const unsigned char *>(k_new);
+    p.v_new = static_cast<const unsigned char *>(v_new);
+    p.slots = slot_mapping_dev;
+    p.n_tokens = n_tokens;
+    p.block_size = pool->cfg.block_size;
+    p.num_kv_heads = pool->cfg.num_kv_heads;
+    p.row_chunks = (int32_t)(row_bytes / 16);
+    p.num_blocks = pool->cfg.num_blocks;
+    const int grid = n_tokens < 148 * 32 ? n_tokens : 148 * 32;
+    append_kv_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    pa_internal::launch_count.fetch_add(1);
+    return check_launch("append_kv_kernel");
+}
+
+pa_status pa_copy_blocks(pa_pool *pool, const int32_t *pairs_dev, int32_t n_pairs, pa_stream stream) {
+    if (!pool || !pool->k_pool) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: pool has no device memory");
+    if (n_pairs < 0) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: negative n_pairs");
+    if (n_pairs == 0) return PA_OK;
+    if (!pairs_dev || ((uintptr_t)pairs_dev & 3)) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: bad pairs pointer");
+    if (pool->block_bytes() % 16) return fail(PA_ERR_UNSUPPORTED, "pa_copy_blocks: block bytes not a multiple of 16");
+    if (pool->cfg.num_layers > 65535) return fail(PA_ERR_UNSUPPORTED, "pa_copy_blocks: too many layers");
+    CopyParams p;
+    p.k_pool = static_cast<unsigned char *>(pool->k_pool);
+    p.v_pool = static_cast<unsigned char *>(pool->v_pool);
+    p.pairs = pairs_dev;
+    p.block_chunks = (int64_t)(pool->block_bytes() / 16);
+    p.layer_chunks = (int64_t)(pool->layer_bytes() / 16);
+    p.num_blocks = pool->cfg.num_blocks;
+    copy_blocks_kernel<<<dim3(n_pairs, pool->cfg.num_layers, 2), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    pa_internal::launch_count.fetch_add(1);
+    return check_launch("copy_blocks_kernel");
+}
+
+pa_status pa_device_error(int32_t *code, int32_t clear) {
+    if (!code) return fail(PA_ERR_INVALID_ARG, "pa_device_error: null code");
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof v);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("pa_device_error: ") + cudaGetErrorString(e));
+    *code = (int32_t)v;
+    if (clear) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("pa_device_error: ") + cudaGetErrorString(e));
+    }
+    return PA_OK;
+}
+
+}  // extern "C"

@@ -73,13 +73,18 @@ def continuous_schedule(n: int, steps: int, seed: int, lo: int = 128, hi: int = 
     return ContinuousSchedule(initial=initial, events=events)
 
 
-def continuous_batch(seed: int = 3, n: int = 256, steps: int = 64) -> dict:
-    """256 sequences, lengths U[128, 4096], block 16, 32 q / 8 KV heads, d128, bf16."""
+def continuous_batch(seed: int = 3, n: int = 256, steps: int = 64, p_stop: float = 1.0 / 200.0,
+                     lo: int = 128, hi: int = 4096) -> dict:
+    """256 sequences, lengths U[128, 4096], block 16, 32 q / 8 KV heads, d128, bf16.
+
+    Pool: every slot can hold a maximum-length sequence plus the steps' appends, so
+    the pool never runs out (n * ceil((hi + steps) / 16) blocks; 66,560 at the
+    default sizes)."""
     shape = Shape(1, 16, 32, 8, 128, "bf16",
-                  num_blocks=n * ((4096 + 64 + 15) // 16), kv_scale=1.0 / math.sqrt(128.0))
+                  num_blocks=n * ((hi + max(steps, 64) + 15) // 16), kv_scale=1.0 / math.sqrt(128.0))
     order = np.random.default_rng(seed + 1000).permutation(shape.num_blocks).astype(np.int32)
     return dict(name="continuous_batch", seed=seed, shape=shape, order=order,
-                schedule=continuous_schedule(n, steps, seed))
+                schedule=continuous_schedule(n, steps, seed, lo, hi, p_stop))
 
 
 def prefix_sharing(seed: int = 4, n: int = 64, prefix: int = 2048) -> dict:

@@ -16,3 +16,12 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+def pytest_sessionstart(session):
+    # Build (or refresh) the native libraries once per session; nvcc cross-compiles
+    # sm_100a without a GPU.  Nothing falls back if this fails.
+    from paged_kv_cache_403_b200 import build
+    import oracle.build
+    build.build_all()
+    oracle.build.build()

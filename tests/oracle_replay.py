@@ -1,0 +1,104 @@
+"""Replays a workload on the oracle side (test helper; imports only oracle/ and synthetic/).
+
+Inputs are regenerated on the host from the seeded generators; nothing here reads
+data produced by the CUDA path.  Expected outputs come from oracle.paged_decode.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+import oracle
+from oracle.block_manager import BlockManagerModel
+from oracle.cache_model import append_rows, copy_blocks, empty_pools
+from synthetic import values as sv
+
+TOL = {"f32": 1e-5, "f16": 2e-3, "bf16": 2e-3}   # max-abs, fp32 output
+ULP = {"f32": 2.0 ** -23, "f16": 2.0 ** -10, "bf16": 2.0 ** -7}
+
+
+def narrow_bound(ref: np.ndarray, out_dtype: str, kv_dtype: str) -> np.ndarray:
+    """Allowed |gpu - oracle| when the result is stored in `out_dtype`: the arithmetic
+    tolerance plus half an ulp of the output format at the reference value."""
+    mag = np.maximum(np.abs(ref), 2.0 ** -14)
+    ulp = ULP[out_dtype] * 2.0 ** np.floor(np.log2(mag))
+    return TOL[kv_dtype] + (0.5 * ulp if out_dtype != "f32" else 0.0)
+
+
+def check_close(gpu: np.ndarray, ref: np.ndarray, out_dtype: str, kv_dtype: str, what: str = ""):
+    err = np.abs(gpu.astype(np.float64) - ref)
+    bound = narrow_bound(ref, out_dtype, kv_dtype)
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {bad.sum()} elements over tolerance; max err {err.max():.3g} "
+                           f"at {np.unravel_index(err.argmax(), err.shape)}")
+    return float(err.max())
+
+
+class OracleRun:
+    """Oracle-side mirror: block manager model + host pools + fp64 attention."""
+
+    def __init__(self, shape, order, seed):
+        self.shape, self.seed = shape, seed
+        self.bm = BlockManagerModel(shape.num_blocks, shape.block_size, order)
+        self.k, self.v = empty_pools(shape.num_layers, shape.num_blocks, shape.num_kv_heads,
+                                     shape.block_size, shape.head_dim, shape.dtype)
+
+    def rows(self, kind, layer, uids, toks):
+        s = self.shape
+        heads = s.num_q_heads if kind == sv.KIND_Q else s.num_kv_heads
+        scale = s.q_scale if kind == sv.KIND_Q else s.kv_scale
+        return sv.rows(kind, self.seed, layer, uids, toks, heads, s.head_dim, scale, s.dtype)
+
+    def write(self, slots, uids, toks):
+        for layer in range(self.shape.num_layers):
+            append_rows(self.k, self.v, layer, slots, self.rows(sv.KIND_K, layer, uids, toks),
+                        self.rows(sv.KIND_V, layer, uids, toks))
+
+    def prefill(self, sids, uids, lens):
+        slots, cow = self.bm.reserve_slots(sids, lens)
+        assert not cow
+        self.write(slots, np.repeat(uids, lens), np.concatenate([np.arange(L) for L in lens]))
+        return slots
+
+    def decode_step(self, sids, uids, max_blocks, layers=None):
+        positions = [self.bm.length(s) for s in sids]
+        slots, cow = self.bm.reserve_slots(sids, [1] * len(sids))
+        copy_blocks(self.k, self.v, cow)
+        self.write(slots, uids, positions)
+        tables, lens = self.bm.dense_tables(sids, max_blocks)
+        tables = np.array(tables, np.int32)
+        lens = np.array(lens, np.int32)
+        outs = {}
+        for layer in (range(self.shape.num_layers) if layers is None else layers):
+            q = self.rows(sv.KIND_Q, layer, uids, positions)
+            outs[layer] = oracle.paged_decode(self.k[layer], self.v[layer], self.shape.dtype, tables, lens, q,
+                                              1.0 / math.sqrt(self.shape.head_dim))
+        return dict(slots=np.array(slots, np.int64), cow=np.array(cow, np.int32).reshape(-1, 2),
+                    tables=tables, lens=lens, outputs=outs, positions=np.array(positions))
+
+
+def sequence_attention(shape, seed, layer, uid, length, q_uid, q_pos, writer=None):
+    """fp64 attention of one query against one sequence's regenerated history.
+
+    writer(pos) -> (uid, token) names who wrote position pos (default: uid, pos).
+    The history is laid into a contiguous pool with an identity block table.
+    """
+    B, hkv, d = shape.block_size, shape.num_kv_heads, shape.head_dim
+    pos = np.arange(length)
+    if writer is None:
+        wu, wt = np.full(length, uid), pos
+    else:
+        wu, wt = map(np.array, zip(*[writer(p) for p in pos]))
+    k = sv.rows(sv.KIND_K, seed, layer, wu, wt, hkv, d, shape.kv_scale, shape.dtype)
+    v = sv.rows(sv.KIND_V, seed, layer, wu, wt, hkv, d, shape.kv_scale, shape.dtype)
+    nblk = -(-length // B)
+    pad = nblk * B - length
+    if pad:
+        k = np.concatenate([k, np.zeros((pad, hkv, d), k.dtype)])
+        v = np.concatenate([v, np.zeros((pad, hkv, d), v.dtype)])
+    kp = np.ascontiguousarray(k.reshape(nblk, B, hkv, d).transpose(0, 2, 1, 3))
+    vp = np.ascontiguousarray(v.reshape(nblk, B, hkv, d).transpose(0, 2, 1, 3))
+    q = sv.rows(sv.KIND_Q, seed, layer, [q_uid], [q_pos], shape.num_q_heads, d, shape.q_scale, shape.dtype)
+    return oracle.paged_decode(kp, vp, shape.dtype, np.arange(nblk, dtype=np.int32)[None], np.array([length]),
+                               q, 1.0 / math.sqrt(d))[0]
