@@ -1,6 +1,6 @@
 // sm_100a kernels of the paged decode path and their C ABI entry points.
 //
-//  paged_decode_kernel  -- single-query decode attention through the block
+//  paged_decode_simt_kernel  -- single-query decode attention through the block
 //                          table ("What problem does PagedAttention solve, and
 //                          what is continuous batching?", "How PagedAttention
 //                          works": the kernel follows the table when it reads
@@ -28,6 +28,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cmath>
 #include <cstdint>
@@ -238,7 +239,7 @@ __device__ __forceinline__ void store_out(const DecodeParams &p, size_t idx, flo
 }
 
 template <typename T, int B, int D, int HPC>
-__global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kDecodeThreads) paged_decode_simt_kernel(const DecodeParams p) {
     using EL = Elem<T>;
     using SH = DecodeShape<T, B, D>;
     constexpr int VEC = SH::kVec, E = SH::kElems, NCH = SH::kChunks, ROW = SH::kRowBytes;
@@ -474,8 +475,16 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const Deco
 }
 
 // ------------------------------------------------------------------ split reduce
+struct ReduceParams {
+    const int32_t *lens;
+    void *out;
+    const float *ws_acc;
+    const float *ws_ml;
+    int32_t max_blocks, num_q_heads, split_blocks, max_splits, out_f32;
+};
+
 template <typename T, int B, int D>
-__global__ void __launch_bounds__(D) split_reduce_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(D) split_reduce_kernel(const ReduceParams p) {
     const int s = blockIdx.x;
     const int hq = blockIdx.y;
     const int d = threadIdx.x;
@@ -495,7 +504,363 @@ __global__ void __launch_bounds__(D) split_reduce_kernel(const DecodeParams p) {
         lsum += p.ws_ml[part * 2 + 1] * f;
         osum += p.ws_acc[part * D + d] * f;
     }
-    store_out<T>(p, ((size_t)s * p.num_q_heads + hq) * D + d, osum / lsum);
+    const float v = osum / lsum;
+    const size_t idx = ((size_t)s * p.num_q_heads + hq) * D + d;
+    if (p.out_f32)
+        static_cast<float *>(p.out)[idx] = v;
+    else
+        static_cast<T *>(p.out)[idx] = Elem<T>::narrow(v);
+}
+
+// ------------------------------------------------------------------ tensor-core decode (fp16 / bf16)
+// Per consumer warp and per 16-token group of a tile:
+//   S^T[16 tok][8 heads]  = K[16][D] . Q^T[D][8]       mma.m16n8k16, K rows via ldmatrix
+//   online softmax down the columns of S^T (one column per query head)
+//   O^T[D][8 heads]      += V^T[D][16] . P^T[16][8]     mma.m16n8k16, V via ldmatrix.trans,
+//                                                       P^T from S^T's layout by movmatrix.trans
+// Query heads beyond the GQA group are zero columns.  P enters the second product as
+// a hi + lo pair of 16-bit halves, so the weights keep about 16 bits.  K and V tiles
+// arrive by 2-D TMA tensor loads with 128-byte swizzle (16-byte chunk c of row r sits
+// at chunk c ^ (r % 8) of a 128-byte row), which makes the ldmatrix reads free of
+// bank conflicts.
+template <typename T>
+struct Mma;
+
+template <>
+struct Mma<__nv_bfloat16> {
+    __device__ __forceinline__ static void mma(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    // two floats -> one register, `lo` in the low half
+    __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+        uint32_t r;
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+        return r;
+    }
+    __device__ __forceinline__ static float low(uint32_t r) { return __uint_as_float(r << 16); }
+    __device__ __forceinline__ static float high(uint32_t r) { return __uint_as_float(r & 0xffff0000u); }
+};
+
+template <>
+struct Mma<__half> {
+    __device__ __forceinline__ static void mma(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+        uint32_t r;
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+        return r;
+    }
+    __device__ __forceinline__ static float low(uint32_t r) {
+        return __half2float(__ushort_as_half((unsigned short)(r & 0xffffu)));
+    }
+    __device__ __forceinline__ static float high(uint32_t r) {
+        return __half2float(__ushort_as_half((unsigned short)(r >> 16)));
+    }
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
+    uint32_t r;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+    return r;
+}
+
+// 2-D TMA tensor load (no multicast) completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+struct MmaParams {
+    CUtensorMap tmap_k;             // [L*NB*Hkv*B rows][D] key pool
+    CUtensorMap tmap_v;
+    const void *q;
+    void *out;
+    const int32_t *tables;
+    const int32_t *lens;
+    float *ws_acc;
+    float *ws_ml;
+    int32_t max_blocks, num_blocks, num_kv_heads, num_q_heads, layer;
+    int32_t split_blocks, max_splits, out_f32, heads_per_cta;
+    float scale_log2;
+};
+
+template <int B, int D>
+struct MmaShape {
+    static constexpr int kBoxes = D / 64;                 // 128-byte column boxes per row
+    static constexpr int kBoxBytes = B * 128;             // one box: B rows x 128 bytes
+    static constexpr int kTileBytes = kBoxes * kBoxBytes;  // B x D x 2 bytes
+    static constexpr int kStages = (2 * kTileBytes <= 8192) ? 8 : 4;
+    static constexpr int kRingBytes = kStages * 2 * kTileBytes;
+    static constexpr int kRedBytes = kConsumerWarps * 8 * (2 + D) * 4;
+    static_assert(kRedBytes <= kRingBytes, "reduction area reuses the ring");
+    static_assert(kStages % kConsumerWarps == 0, "each stage must belong to one consumer warp");
+    static constexpr size_t kSmemBytes = 1024 + kRingBytes + 2 * kStages * sizeof(uint64_t);
+};
+
+template <typename T, int B, int D>
+__global__ void __launch_bounds__(kDecodeThreads, 3) paged_decode_mma_kernel(const __grid_constant__ MmaParams p) {
+    using SH = MmaShape<B, D>;
+    using M = Mma<T>;
+    constexpr int STAGES = SH::kStages, TILE = SH::kTileBytes, BOX = SH::kBoxBytes, KD = D / 16;
+    extern __shared__ unsigned char smem_raw[];
+    // 128-byte swizzled TMA destinations want 1024-byte alignment
+    unsigned char *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+
+    const int s = blockIdx.x;
+    const int hg = blockIdx.y;
+    const int split = blockIdx.z;
+    const int hpc = p.heads_per_cta;
+
+    int L = p.lens[s];
+    if (L < 1 || (L + B - 1) / B > p.max_blocks) {
+        if (threadIdx.x == 0 && hg == 0 && split == 0) raise_error(kErrBadLen);
+        if (L < 1) {
+            if (split == 0)
+                for (int t = threadIdx.x; t < hpc * D; t += blockDim.x) {
+                    const size_t idx = ((size_t)s * p.num_q_heads + hg * hpc + t / D) * D + t % D;
+                    if (p.out_f32)
+                        static_cast<float *>(p.out)[idx] = 0.f;
+                    else
+                        static_cast<T *>(p.out)[idx] = Elem<T>::narrow(0.f);
+                }
+            return;
+        }
+        L = p.max_blocks * B;
+    }
+    const int nblk = (L + B - 1) / B;
+    const int b0 = split * p.split_blocks;
+    if (b0 >= nblk) return;
+    const int ntiles = min(nblk, b0 + p.split_blocks) - b0;
+    const int nsplit = (nblk + p.split_blocks - 1) / p.split_blocks;
+    const int group = p.num_q_heads / p.num_kv_heads;
+    const int h0 = hg * hpc;
+    const int g = h0 / group;
+
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + SH::kRingBytes);
+    uint64_t *empty = full + STAGES;
+    float *red_m = reinterpret_cast<float *>(smem);               // [warps][8], after the loop
+    float *red_l = red_m + kConsumerWarps * 8;                     // [warps][8]
+    float *red_o = red_l + kConsumerWarps * 8;                     // [warps][8][D]
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_fence_init();
+    }
+    __syncthreads();
+
+    const int gq = lane >> 2;   // accumulator row group
+    const int tq = lane & 3;    // accumulator column pair
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads 2tq, 2tq+1
+    float o[KD][4];
+
+    if (warp == kConsumerWarps) {
+        // ---------------- producer
+        const int32_t *trow = p.tables + (size_t)s * p.max_blocks + b0;
+        bool ok = true;
+        for (int base = 0; base < ntiles && ok; base += 32) {
+            int blk = 0;
+            if (base + lane < ntiles) {
+                blk = trow[base + lane];
+                if ((unsigned)blk >= (unsigned)p.num_blocks) {
+                    raise_error(kErrBadBlock);
+                    blk = 0;
+                }
+            }
+            const int cnt = min(32, ntiles - base);
+            for (int j = 0; j < cnt; ++j) {
+                const int b = __shfl_sync(0xffffffffu, blk, j);
+                const int i = base + j;
+                const int st = i % STAGES;
+                if (lane == 0) {
+                    if (i >= STAGES) ok = mbar_wait_thread(&empty[st], ((i / STAGES) - 1) & 1);
+                    if (ok) {
+                        const int row = ((p.layer * p.num_blocks + b) * p.num_kv_heads + g) * B;
+                        unsigned char *dst = smem + st * 2 * TILE;
+                        mbar_arrive_expect_tx(&full[st], 2 * TILE);
+#pragma unroll
+                        for (int bx = 0; bx < SH::kBoxes; ++bx) {
+                            tma_load_2d(dst + bx * BOX, &p.tmap_k, bx * 64, row, &full[st]);
+                            tma_load_2d(dst + TILE + bx * BOX, &p.tmap_v, bx * 64, row, &full[st]);
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+            }
+        }
+    } else {
+        // ---------------- consumers
+        uint32_t qb[KD][2];   // Q^T fragments: column gq is query head h0 + gq
+        {
+            const bool qv = gq < hpc;
+            const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
+                static_cast<const T *>(p.q) + ((size_t)s * p.num_q_heads + h0 + (qv ? gq : 0)) * D);
+#pragma unroll
+            for (int kk = 0; kk < KD; ++kk) {
+                qb[kk][0] = qv ? qrow[(kk * 16 + 2 * tq) / 2] : 0u;
+                qb[kk][1] = qv ? qrow[(kk * 16 + 8 + 2 * tq) / 2] : 0u;
+            }
+        }
+#pragma unroll
+        for (int dm = 0; dm < KD; ++dm) o[dm][0] = o[dm][1] = o[dm][2] = o[dm][3] = 0.f;
+        const float sl = p.scale_log2;
+
+        for (int i = warp; i < ntiles; i += kConsumerWarps) {
+            const int st = i % STAGES;
+            if (!mbar_wait_warp(&full[st], (i / STAGES) & 1)) break;
+            const uint32_t kbase = smem_addr(smem + st * 2 * TILE);
+            const uint32_t vbase = kbase + TILE;
+            const int tok0 = (b0 + i) * B;
+#pragma unroll
+            for (int j = 0; j < B / 16; ++j) {
+                if (tok0 + j * 16 >= L) break;          // nothing valid in this group
+                float c[4] = {0.f, 0.f, 0.f, 0.f};
+                {
+                    const int r = j * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+                    for (int kk = 0; kk < KD; ++kk) {
+                        const int chunk = (kk & 3) * 2 + (lane >> 4);
+                        uint32_t a[4];
+                        ldsm_x4(a, kbase + (kk >> 2) * BOX + r * 128 + ((chunk ^ (r & 7)) << 4));
+                        M::mma(c, a, qb[kk][0], qb[kk][1]);
+                    }
+                }
+                const bool v0 = tok0 + j * 16 + gq < L;
+                const bool v1 = tok0 + j * 16 + gq + 8 < L;
+                const float s0 = v0 ? c[0] * sl : -INFINITY, s1 = v0 ? c[1] * sl : -INFINITY;
+                const float s2 = v1 ? c[2] * sl : -INFINITY, s3 = v1 ? c[3] * sl : -INFINITY;
+                const bool need = fmaxf(s0, s2) > m0 + kRescaleThreshold || fmaxf(s1, s3) > m1 + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, need)) {
+                    float t0 = fmaxf(s0, s2), t1 = fmaxf(s1, s3);
+#pragma unroll
+                    for (int off = 4; off < 32; off <<= 1) {
+                        t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, off));
+                        t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, off));
+                    }
+                    const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
+                    const float f0 = ex2(m0 - n0), f1 = ex2(m1 - n1);
+                    l0 *= f0;
+                    l1 *= f1;
+#pragma unroll
+                    for (int dm = 0; dm < KD; ++dm) {
+                        o[dm][0] *= f0;
+                        o[dm][2] *= f0;
+                        o[dm][1] *= f1;
+                        o[dm][3] *= f1;
+                    }
+                    m0 = n0;
+                    m1 = n1;
+                }
+                const float p0 = ex2(s0 - m0), p1 = ex2(s1 - m1), p2 = ex2(s2 - m0), p3 = ex2(s3 - m1);
+                l0 += p0 + p2;
+                l1 += p1 + p3;
+                const uint32_t h01 = M::pack(p0, p1), h23 = M::pack(p2, p3);
+                const uint32_t r01 = M::pack(p0 - M::low(h01), p1 - M::high(h01));
+                const uint32_t r23 = M::pack(p2 - M::low(h23), p3 - M::high(h23));
+                const uint32_t bh0 = transpose8x8(h01), bh1 = transpose8x8(h23);
+                const uint32_t bl0 = transpose8x8(r01), bl1 = transpose8x8(r23);
+                {
+                    const int mi = lane >> 3;
+                    const int r = j * 16 + (lane & 7) + (mi >> 1) * 8;
+#pragma unroll
+                    for (int dm = 0; dm < KD; ++dm) {
+                        const int chunk = (dm & 3) * 2 + (mi & 1);
+                        uint32_t a[4];
+                        ldsm_x4_trans(a, vbase + (dm >> 2) * BOX + r * 128 + ((chunk ^ (r & 7)) << 4));
+                        M::mma(o[dm], a, bh0, bh1);
+                        M::mma(o[dm], a, bl0, bl1);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        // l: sum over the eight token rows held by lanes differing in bits 2..4
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+        }
+    }
+    __syncthreads();   // every stage consumed and every copy landed: the ring is free
+    if (warp < kConsumerWarps) {
+        if (gq == 0) {
+            red_m[warp * 8 + 2 * tq] = m0;
+            red_m[warp * 8 + 2 * tq + 1] = m1;
+            red_l[warp * 8 + 2 * tq] = l0;
+            red_l[warp * 8 + 2 * tq + 1] = l1;
+        }
+#pragma unroll
+        for (int dm = 0; dm < KD; ++dm) {
+            float *c0 = red_o + (warp * 8 + 2 * tq) * D + dm * 16 + gq;
+            float *c1 = c0 + D;
+            c0[0] = o[dm][0];
+            c1[0] = o[dm][1];
+            c0[8] = o[dm][2];
+            c1[8] = o[dm][3];
+        }
+    }
+    __syncthreads();
+
+    for (int t = threadIdx.x; t < hpc * D; t += blockDim.x) {
+        const int h = t / D;
+        const int d = t % D;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, red_m[w * 8 + h]);
+        float lsum = 0.f, osum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+            const float mw = red_m[w * 8 + h];
+            const float f = (mw == -INFINITY) ? 0.f : ex2(mw - mx);
+            lsum += red_l[w * 8 + h] * f;
+            osum += red_o[(w * 8 + h) * D + d] * f;
+        }
+        const int hq = h0 + h;
+        if (nsplit == 1) {
+            const size_t idx = ((size_t)s * p.num_q_heads + hq) * D + d;
+            if (p.out_f32)
+                static_cast<float *>(p.out)[idx] = osum / lsum;
+            else
+                static_cast<T *>(p.out)[idx] = Elem<T>::narrow(osum / lsum);
+        } else {
+            const size_t part = ((size_t)s * p.max_splits + split) * p.num_q_heads + hq;
+            p.ws_acc[part * D + d] = osum;
+            if (d == 0) {
+                p.ws_ml[part * 2] = mx;
+                p.ws_ml[part * 2 + 1] = lsum;
+            }
+        }
+    }
 }
 
 // ------------------------------------------------------------------ append / copy
@@ -575,40 +940,105 @@ pa_status ensure_smem(K kernel, size_t bytes, bool (&done)[64]) {
     return PA_OK;
 }
 
+template <typename T, int B, int D>
+pa_status launch_reduce(const ReduceParams &r, int n_seqs, cudaStream_t stream) {
+    if (r.max_splits <= 1) return PA_OK;
+    split_reduce_kernel<T, B, D><<<dim3(n_seqs, r.num_q_heads), D, 0, stream>>>(r);
+    pa_internal::launch_count.fetch_add(1);
+    return check_launch("split_reduce_kernel");
+}
+
 template <typename T, int B, int D, int HPC>
-pa_status launch_decode(const DecodeParams &p, cudaStream_t stream) {
+pa_status launch_simt(const DecodeParams &p, const ReduceParams &r, cudaStream_t stream) {
     constexpr size_t smem = decode_smem_bytes<T, B, D, HPC>();
-    auto kernel = paged_decode_kernel<T, B, D, HPC>;
+    auto kernel = paged_decode_simt_kernel<T, B, D, HPC>;
     static bool smem_set[64] = {};
     pa_status st = ensure_smem(kernel, smem, smem_set);
     if (st != PA_OK) return st;
     dim3 grid(p.n_seqs, p.num_q_heads / HPC, p.max_splits);
     kernel<<<grid, kDecodeThreads, smem, stream>>>(p);
     pa_internal::launch_count.fetch_add(1);
-    st = check_launch("paged_decode_kernel");
-    if (st != PA_OK || p.max_splits <= 1) return st;
-    split_reduce_kernel<T, B, D><<<dim3(p.n_seqs, p.num_q_heads), D, 0, stream>>>(p);
-    pa_internal::launch_count.fetch_add(1);
-    return check_launch("split_reduce_kernel");
+    st = check_launch("paged_decode_simt_kernel");
+    if (st != PA_OK) return st;
+    return launch_reduce<T, B, D>(r, p.n_seqs, stream);
 }
 
 template <typename T, int B, int D>
-pa_status dispatch_hpc(const DecodeParams &p, int hpc, cudaStream_t stream) {
+pa_status dispatch_hpc(const DecodeParams &p, const ReduceParams &r, int hpc, cudaStream_t stream) {
     switch (hpc) {
-    case 1: return launch_decode<T, B, D, 1>(p, stream);
-    case 2: return launch_decode<T, B, D, 2>(p, stream);
-    case 4: return launch_decode<T, B, D, 4>(p, stream);
+    case 1: return launch_simt<T, B, D, 1>(p, r, stream);
+    case 2: return launch_simt<T, B, D, 2>(p, r, stream);
+    case 4: return launch_simt<T, B, D, 4>(p, r, stream);
     }
     return fail(PA_ERR_UNSUPPORTED, "unsupported query heads per KV head");
 }
 
 template <typename T>
-pa_status dispatch_shape(const DecodeParams &p, int B, int D, int hpc, cudaStream_t stream) {
-    if (B == 16 && D == 128) return dispatch_hpc<T, 16, 128>(p, hpc, stream);
-    if (B == 32 && D == 128) return dispatch_hpc<T, 32, 128>(p, hpc, stream);
-    if (B == 16 && D == 64) return dispatch_hpc<T, 16, 64>(p, hpc, stream);
-    if (B == 32 && D == 64) return dispatch_hpc<T, 32, 64>(p, hpc, stream);
+pa_status dispatch_simt(const DecodeParams &p, const ReduceParams &r, int B, int D, int hpc, cudaStream_t stream) {
+    if (B == 16 && D == 128) return dispatch_hpc<T, 16, 128>(p, r, hpc, stream);
+    if (B == 32 && D == 128) return dispatch_hpc<T, 32, 128>(p, r, hpc, stream);
+    if (B == 16 && D == 64) return dispatch_hpc<T, 16, 64>(p, r, hpc, stream);
+    if (B == 32 && D == 64) return dispatch_hpc<T, 32, 64>(p, r, hpc, stream);
     return fail(PA_ERR_UNSUPPORTED, "block_size must be 16 or 32 and head_dim 64 or 128");
+}
+
+template <typename T, int B, int D>
+pa_status launch_mma(const MmaParams &p, const ReduceParams &r, int n_seqs, cudaStream_t stream) {
+    constexpr size_t smem = MmaShape<B, D>::kSmemBytes;
+    auto kernel = paged_decode_mma_kernel<T, B, D>;
+    static bool smem_set[64] = {};
+    pa_status st = ensure_smem(kernel, smem, smem_set);
+    if (st != PA_OK) return st;
+    dim3 grid(n_seqs, p.num_q_heads / p.heads_per_cta, p.max_splits);
+    kernel<<<grid, kDecodeThreads, smem, stream>>>(p);
+    pa_internal::launch_count.fetch_add(1);
+    st = check_launch("paged_decode_mma_kernel");
+    if (st != PA_OK) return st;
+    return launch_reduce<T, B, D>(r, n_seqs, stream);
+}
+
+template <typename T>
+pa_status dispatch_mma(const MmaParams &p, const ReduceParams &r, int n_seqs, int B, int D, cudaStream_t stream) {
+    if (B == 16 && D == 128) return launch_mma<T, 16, 128>(p, r, n_seqs, stream);
+    if (B == 32 && D == 128) return launch_mma<T, 32, 128>(p, r, n_seqs, stream);
+    if (B == 16 && D == 64) return launch_mma<T, 16, 64>(p, r, n_seqs, stream);
+    if (B == 32 && D == 64) return launch_mma<T, 32, 64>(p, r, n_seqs, stream);
+    return fail(PA_ERR_UNSUPPORTED, "block_size must be 16 or 32 and head_dim 64 or 128");
+}
+
+// TMA descriptors over a 16-bit pool: 2-D [rows][head_dim], boxes of 64 elements
+// (128 bytes, the 128-byte swizzle span) by block_size rows.
+pa_status ensure_tensor_maps(pa_pool *pool) {
+    if (pool->tmaps_ready) return PA_OK;
+    using Encode = PFN_cuTensorMapEncodeTiled_v12000;
+    static Encode encode = nullptr;
+    if (!encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+        encode = reinterpret_cast<Encode>(fn);
+    }
+    const pa_pool_config &c = pool->cfg;
+    const uint64_t rows = (uint64_t)c.num_layers * c.num_blocks * c.num_kv_heads * c.block_size;
+    if (rows >= (1ull << 31))
+        return fail(PA_ERR_UNSUPPORTED, "pool too large for 32-bit TMA row coordinates");
+    const CUtensorMapDataType dt = c.dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    cuuint64_t dims[2] = {(cuuint64_t)c.head_dim, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)c.head_dim * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)c.block_size};
+    cuuint32_t estr[2] = {1, 1};
+    void *bases[2] = {pool->k_pool, pool->v_pool};
+    CUtensorMap *maps[2] = {&pool->tmap_k, &pool->tmap_v};
+    for (int i = 0; i < 2; ++i) {
+        CUresult r = encode(maps[i], dt, 2, bases[i], dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")");
+    }
+    pool->tmaps_ready = true;
+    return PA_OK;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -655,41 +1085,77 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
     if (split_tokens < 0 || (split_tokens > 0 && split_tokens % c.block_size != 0))
         return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: split_tokens must be 0 or a multiple of block_size");
     const int32_t max_splits = pa_decode_max_splits(c.block_size, max_blocks, split_tokens);
-    const int hpc = group < 4 ? group : 4;
-    if (max_splits > 65535 || num_q_heads / hpc > 65535)
+    if (max_splits > 65535 || num_q_heads > 65535)
         return fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: grid too large");
     const size_t need = pa_decode_workspace_bytes(n_seqs, num_q_heads, c.head_dim, max_splits);
     if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
         return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: workspace missing, misaligned or smaller than " +
                                             std::to_string(need) + " bytes");
 
-    DecodeParams p;
-    p.k_layer = static_cast<const unsigned char *>(pool->k_pool) + (size_t)layer * pool->layer_bytes();
-    p.v_layer = static_cast<const unsigned char *>(pool->v_pool) + (size_t)layer * pool->layer_bytes();
+    const size_t parts = (size_t)n_seqs * max_splits * num_q_heads;
+    float *ws_acc = static_cast<float *>(workspace);
+    float *ws_ml = need > 0 ? static_cast<float *>(workspace) + parts * c.head_dim : nullptr;
+    const int32_t split_blocks = split_tokens > 0 ? split_tokens / c.block_size : max_blocks;
+    const float scale_log2 = (float)((double)scale * 1.4426950408889634);   // scale * log2(e)
+
+    ReduceParams r;
+    r.lens = seq_lens_dev;
+    r.out = out;
+    r.ws_acc = ws_acc;
+    r.ws_ml = ws_ml;
+    r.max_blocks = max_blocks;
+    r.num_q_heads = num_q_heads;
+    r.split_blocks = split_blocks;
+    r.max_splits = max_splits;
+    r.out_f32 = out_dtype == PA_F32;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (c.dtype == PA_F32) {
+        // fp32 caches: CUDA-core kernel (the tensor-core path takes 16-bit operands only)
+        DecodeParams p;
+        p.k_layer = static_cast<const unsigned char *>(pool->k_pool) + (size_t)layer * pool->layer_bytes();
+        p.v_layer = static_cast<const unsigned char *>(pool->v_pool) + (size_t)layer * pool->layer_bytes();
+        p.q = q;
+        p.out = out;
+        p.tables = block_tables_dev;
+        p.lens = seq_lens_dev;
+        p.ws_acc = ws_acc;
+        p.ws_ml = ws_ml;
+        p.n_seqs = n_seqs;
+        p.max_blocks = max_blocks;
+        p.num_blocks = c.num_blocks;
+        p.num_kv_heads = c.num_kv_heads;
+        p.num_q_heads = num_q_heads;
+        p.split_blocks = split_blocks;
+        p.max_splits = max_splits;
+        p.out_f32 = r.out_f32;
+        p.scale_log2 = scale_log2;
+        const int hpc = group < 4 ? group : 4;
+        return dispatch_simt<float>(p, r, c.block_size, c.head_dim, hpc, st);
+    }
+    pa_status s2 = ensure_tensor_maps(pool);
+    if (s2 != PA_OK) return s2;
+    MmaParams p;
+    p.tmap_k = pool->tmap_k;
+    p.tmap_v = pool->tmap_v;
     p.q = q;
     p.out = out;
     p.tables = block_tables_dev;
     p.lens = seq_lens_dev;
-    const size_t parts = (size_t)n_seqs * max_splits * num_q_heads;
-    p.ws_acc = static_cast<float *>(workspace);
-    p.ws_ml = need > 0 ? static_cast<float *>(workspace) + parts * c.head_dim : nullptr;
-    p.n_seqs = n_seqs;
+    p.ws_acc = ws_acc;
+    p.ws_ml = ws_ml;
     p.max_blocks = max_blocks;
     p.num_blocks = c.num_blocks;
     p.num_kv_heads = c.num_kv_heads;
     p.num_q_heads = num_q_heads;
-    p.split_blocks = split_tokens > 0 ? split_tokens / c.block_size : max_blocks;
+    p.layer = layer;
+    p.split_blocks = split_blocks;
     p.max_splits = max_splits;
-    p.out_f32 = out_dtype == PA_F32;
-    p.scale_log2 = (float)((double)scale * 1.4426950408889634);   // scale * log2(e)
-
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (c.dtype) {
-    case PA_F32: return dispatch_shape<float>(p, c.block_size, c.head_dim, hpc, st);
-    case PA_F16: return dispatch_shape<__half>(p, c.block_size, c.head_dim, hpc, st);
-    case PA_BF16: return dispatch_shape<__nv_bfloat16>(p, c.block_size, c.head_dim, hpc, st);
-    }
-    return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: unknown dtype");
+    p.out_f32 = r.out_f32;
+    p.heads_per_cta = group;   // the whole GQA group (<= 8) shares one CTA
+    p.scale_log2 = scale_log2;
+    if (c.dtype == PA_BF16) return dispatch_mma<__nv_bfloat16>(p, r, n_seqs, c.block_size, c.head_dim, st);
+    return dispatch_mma<__half>(p, r, n_seqs, c.block_size, c.head_dim, st);
 }
 
 pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const void *v_new,

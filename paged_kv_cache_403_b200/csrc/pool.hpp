@@ -1,6 +1,8 @@
 // Internal definition of the opaque pa_pool and shared host helpers.
 #pragma once
 
+#include <cuda.h>
+
 #include <atomic>
 #include <cstdint>
 #include <string>
@@ -30,6 +32,13 @@ struct pa_pool {
     int32_t num_shared = 0;           // blocks with refcount > 1
     int32_t peak_used = 0;
     int64_t fail_alloc_after = -1;    // host fault injection (< 0: off)
+
+    // TMA descriptors over the whole key / value pools, viewed as 2-D tensors of
+    // [num_layers * num_blocks * num_kv_heads * block_size rows][head_dim]; built on
+    // the first decode call (16-bit caches only).
+    bool tmaps_ready = false;
+    CUtensorMap tmap_k;
+    CUtensorMap tmap_v;
 
     size_t elem_bytes() const { return cfg.dtype == PA_F32 ? 4 : 2; }
     // bytes of one (block, kv-head) tile and of one block across heads
