@@ -46,6 +46,24 @@ def parse():
     return ap.parse_args()
 
 
+def captured_traffic():
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if the
+    kernel source is still the one that was captured (else None)."""
+    import hashlib
+    import re
+    prof = os.path.join(ROOT, "profiles", "decode_mma_continuous_batch.md")
+    src = os.path.join(ROOT, "paged_kv_cache_403_b200", "csrc", "kernels.cu")
+    try:
+        text = open(prof).read()
+        sha = re.search(r"kernels.cu sha256 prefix at capture: ([0-9a-f]+)", text).group(1)
+        gb = float(re.search(r"traffic per launch \(read \+ write\) \| ([0-9.]+) GB", text).group(1))
+    except (OSError, AttributeError):
+        return None
+    if not hashlib.sha256(open(src, "rb").read()).hexdigest().startswith(sha):
+        return None
+    return int(gb * 1e9)
+
+
 # ---------------------------------------------------------------------------- schedule
 def simulate(sched, n, steps):
     """Host-side replay of the schedule: per step the uids, token positions and admissions."""
@@ -122,6 +140,23 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": float(np.median([c for c, _ in self.samples])), "sm_max_mhz": float(self.max_mhz),
                 "samples": len(self.samples), "reasons": sorted(reasons), "source": "nvml"}
+
+
+# ---------------------------------------------------------------------------- ranks
+def combine_ranks(dist, times_ms, byte_counts, device):
+    """Whole-job figures over ranks: each time is the max over ranks (the slowest
+    replica bounds the job), each byte count the sum over ranks."""
+    import torch
+    t = torch.tensor(times_ms, dtype=torch.float64, device=device)
+    b = torch.tensor(byte_counts, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return t.tolist(), b.tolist()
+
+
+def replica_seed(rank: int) -> int:
+    """Each rank runs an independent replica of the workload with its own draws."""
+    return 3 + 100 * rank
 
 
 # ---------------------------------------------------------------------------- our path
@@ -293,7 +328,7 @@ def run_ours(args):
     K, W = args.steps, args.warmup
     e2e = not args.no_e2e
     total = W + K + (K if e2e else 0)
-    recipe = wl.continuous_batch(seed=3 + 100 * rank, steps=total)
+    recipe = wl.continuous_batch(seed=replica_seed(rank), steps=total)
     rep = Replica(torch, recipe, total, args.split, device, W + K if e2e else None)
     torch.cuda.synchronize()
 
@@ -348,12 +383,8 @@ def run_ours(args):
 
     # whole-job numbers: bytes summed over ranks, time = max over ranks
     if world > 1:
-        tt = torch.tensor([ms, e2e_res[0] if e2e_res else 0.0], device=device, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        bb = torch.tensor([kv_bytes, e2e_res[1] if e2e_res else 0], device=device, dtype=torch.float64)
-        dist.all_reduce(bb, op=dist.ReduceOp.SUM)
-        ms, kv_tot = tt[0].item(), bb[0].item()
-        e2e_ms, e2e_kv = tt[1].item(), bb[1].item()
+        (ms, e2e_ms), (kv_tot, e2e_kv) = combine_ranks(
+            dist, [ms, e2e_res[0] if e2e_res else 0.0], [kv_bytes, e2e_res[1] if e2e_res else 0], device)
     else:
         kv_tot = kv_bytes
         e2e_ms, e2e_kv = (e2e_res[0], e2e_res[1]) if e2e_res else (0.0, 0)
@@ -385,7 +416,7 @@ def run_ours(args):
             "kv_gb_per_step": round(kv_tot / K / 1e9 / world, 4),
             "hbm_fraction_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "frac": round(achieved / peak, 4), "traffic": captured_traffic(),
                          "kernel": "paged_decode_mma_kernel (+ split_reduce_kernel)",
                          "attn_ms_mean": round(attn_mean_ms, 4),
                          "alg_bytes_per_launch": int(alg_mean), "peak_source": peak_src},
