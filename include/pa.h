@@ -198,6 +198,35 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
                               int32_t num_q_heads, float scale, int32_t split_tokens,
                               void *workspace, size_t ws_bytes, pa_stream stream);
 
+/* Allocation-free decode attention.  The pages have no counterpart: this entry
+ * exists for callers that cannot allocate device memory -- a serving process
+ * that has already handed almost all of the GPU to its KV-cache pool, a host
+ * whose allocator may not be called on the decode path (cudaMalloc can
+ * synchronise the device and stall every stream), or a plain C embedding with no
+ * allocator of its own.  It computes exactly what pa_decode_attention computes,
+ * with the same arguments minus the workspace: the split-K partials go to a fixed
+ * array of PA_STATIC_WORKSPACE_BYTES inside the library, which every GPU that
+ * loads the library keeps until the process exits.
+ *  - It allocates nothing and frees nothing.  The caller still owns q, out, the
+ *    tables, the lengths and the pools.
+ *  - A batch whose partials would not fit, i.e. pa_decode_workspace_bytes(n_seqs,
+ *    num_q_heads, head_dim, pa_decode_max_splits(block_size, max_blocks,
+ *    split_tokens)) > PA_STATIC_WORKSPACE_BYTES, is rejected with
+ *    PA_ERR_INVALID_ARG and a message naming both sizes; nothing is launched.
+ *  - The first call on a device looks up the array's device address with that
+ *    device current and keeps it; make that first call before any stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents.  Nothing in it needs to start at zero (every partial a call reads
+ *    was written earlier in the same call), but calls that overlap on the GPU --
+ *    on different streams, or from different host threads -- race on it and must
+ *    be serialised by the caller. */
+#define PA_STATIC_WORKSPACE_BYTES (16u << 20)
+pa_status pa_decode_attention_static(pa_pool *pool, int32_t layer, const void *q, void *out,
+                                     pa_dtype out_dtype, const int32_t *block_tables_dev,
+                                     int32_t max_blocks, const int32_t *seq_lens_dev,
+                                     int32_t n_seqs, int32_t num_q_heads, float scale,
+                                     int32_t split_tokens, pa_stream stream);
+
 /* ------------------------------------------------------------------ diagnostics */
 
 /* Device error bits recorded by kernels since the last clear (synchronises the

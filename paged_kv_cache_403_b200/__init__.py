@@ -223,6 +223,20 @@ def pa_decode_attention(pool, layer: int, q, out, block_tables_dev, seq_lens_dev
                                       _stream(stream)))
 
 
+PA_STATIC_WORKSPACE_BYTES = 16 << 20
+
+
+def pa_decode_attention_static(pool, layer: int, q, out, block_tables_dev, seq_lens_dev, scale: float,
+                               split_tokens: int = 0, n_seqs=None, stream=None) -> None:
+    """pa_decode_attention without a caller workspace: the split partials live in a
+    fixed array inside the library, so the call allocates no device memory."""
+    n = q.shape[0] if n_seqs is None else n_seqs
+    _check(_lib().pa_decode_attention_static(pool, layer, _dev_ptr(q), _dev_ptr(out), _dtype_code(out.dtype),
+                                             _dev_ptr(block_tables_dev), block_tables_dev.shape[1],
+                                             _dev_ptr(seq_lens_dev), n, q.shape[1], float(scale), split_tokens,
+                                             _stream(stream)))
+
+
 # ------------------------------------------------------------------ diagnostics
 def pa_device_error(clear: bool = False) -> int:
     code = ctypes.c_int32()

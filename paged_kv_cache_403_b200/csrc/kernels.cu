@@ -1045,6 +1045,37 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 }  // namespace
 
+// ------------------------------------------------------------------ allocation-free decode
+// Split-K scratch for pa_decode_attention_static: a fixed array in this library's
+// device memory.  Every GPU that loads the library holds these bytes until the
+// process exits; every call of pa_decode_attention_static on a device shares them.
+static __device__ __align__(256) unsigned char pa_static_split_scratch[PA_STATIC_WORKSPACE_BYTES];
+
+namespace {
+
+// Device address of the scratch array on the current device.  Host code cannot pass
+// the array's name to a kernel (on the host it is only a stand-in symbol), so the
+// first call on each device looks the address up with that device current and
+// keeps it.
+pa_status static_scratch_address(void **out) {
+    static void *addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+    if (dev < 0 || dev >= 64) return fail(PA_ERR_UNSUPPORTED, "pa_decode_attention_static: device ordinal >= 64");
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, pa_static_split_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(PA_ERR_CUDA, std::string("cudaGetSymbolAddress(split scratch): ") + cudaGetErrorString(e));
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return PA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int32_t pa_decode_max_splits(int32_t block_size, int32_t max_blocks, int32_t split_tokens) {
@@ -1203,6 +1234,34 @@ pa_status pa_copy_blocks(pa_pool *pool, const int32_t *pairs_dev, int32_t n_pair
     copy_blocks_kernel<<<dim3(n_pairs, pool->cfg.num_layers, 2), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
     pa_internal::launch_count.fetch_add(1);
     return check_launch("copy_blocks_kernel");
+}
+
+pa_status pa_decode_attention_static(pa_pool *pool, int32_t layer, const void *q, void *out, pa_dtype out_dtype,
+                                     const int32_t *block_tables_dev, int32_t max_blocks, const int32_t *seq_lens_dev,
+                                     int32_t n_seqs, int32_t num_q_heads, float scale, int32_t split_tokens,
+                                     pa_stream stream) {
+    if (!pool) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention_static: null pool");
+    if (n_seqs < 0 || max_blocks < 1 || split_tokens < 0)
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention_static: bad n_seqs, max_blocks or split_tokens");
+    const int32_t max_splits = pa_decode_max_splits(pool->cfg.block_size, max_blocks, split_tokens);
+    if (max_splits < 1)
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention_static: split_tokens must be 0 or a multiple of block_size");
+    const size_t need = pa_decode_workspace_bytes(n_seqs, num_q_heads, pool->cfg.head_dim, max_splits);
+    if (need > (size_t)PA_STATIC_WORKSPACE_BYTES)
+        return fail(PA_ERR_INVALID_ARG,
+                    "pa_decode_attention_static: this batch needs " + std::to_string(need) +
+                        " bytes of split scratch but the built-in array holds " +
+                        std::to_string((size_t)PA_STATIC_WORKSPACE_BYTES) +
+                        "; use a larger split_tokens (or 0), a smaller batch, or pa_decode_attention with a "
+                        "caller-owned workspace");
+    void *ws = nullptr;
+    if (need > 0) {
+        pa_status st = static_scratch_address(&ws);
+        if (st != PA_OK) return st;
+    }
+    return pa_decode_attention(pool, layer, q, out, out_dtype, block_tables_dev, max_blocks, seq_lens_dev, n_seqs,
+                               num_q_heads, scale, split_tokens, ws, need > 0 ? (size_t)PA_STATIC_WORKSPACE_BYTES : 0,
+                               stream);
 }
 
 pa_status pa_device_error(int32_t *code, int32_t clear) {
