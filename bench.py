@@ -1,18 +1,25 @@
 #!/usr/bin/env python
-"""Benchmark: paged decode attention on the continuous-batch workload.
+"""Benchmark: paged decode attention over a paged KV cache, one decode step at a time.
 
-Workload (one replica per GPU): 256 sequences, prompt lengths uniform in
-[128, 4096], block 16, 32 query / 8 KV heads, head_dim 128, bf16 cache; every step
-each sequence appends one token and attends over its whole cache; after each step
-every sequence stops with probability 1/200 and a new one (prompt length uniform
-in [128, 4096]) takes its slot at the next step.  A timed step runs the whole
-path: admissions (prompt K/V appended), one-slot reservations (host), metadata
-upload, append of the step's K/V, decode attention (+ split-K reduce),
-retirements (host).
+Default workload (one replica per GPU), the one the stated target is quoted on:
+continuous batch -- 256 sequences, prompt lengths uniform in [128, 4096], block 16,
+32 query / 8 KV heads, head_dim 128, bf16 cache, 1 layer; every step each sequence
+appends one token and attends over its whole cache; after each step every sequence
+stops with probability 1/200 and a new one (prompt uniform in [128, 4096]) takes its
+slot at the next step.  ``--workload`` selects the other synthetic workloads (the
+pages' worked example, prefix sharing, the ~100 GB 32-layer large pool with block
+16 or 32).
 
-Prints one JSON line (rank 0).  ``value`` is KV bytes read by decode attention per
-second over the timed steps (whole-job, all ranks); decode tokens/s is reported
-beside it.  ``--impl reference`` times the CPU oracle instead on a bounded sample.
+A timed step runs the whole path: admissions (prompt K/V appended), one-slot
+reservations with the copy-on-write check (host, native), metadata upload, then for
+every layer the append of the step's K/V and decode attention (+ split-K reduce),
+and retirements (host).  Host bookkeeping of step t+1 overlaps the GPU work of step
+t: metadata is staged in pinned buffers and uploaded on a side stream into
+NSETS rotating device buffer sets.
+
+Prints one JSON line (rank 0).  ``value`` = KV bytes read by decode attention per
+second of step time, whole job (all ranks); decode tokens/s beside it.
+``--impl reference`` times the CPU oracle on a bounded sample instead.
 """
 from __future__ import annotations
 
@@ -31,19 +38,30 @@ sys.path.insert(0, ROOT)
 METRIC = "paged decode attention KV-read HBM GB/s (fraction of ~8 TB/s) and decode tokens/s"
 UNIT = "GB/s"
 NOMINAL_HBM_GBS = 8000.0
+WORKLOADS = ("continuous_batch", "large_pool_b16", "large_pool_b32", "worked_example", "prefix_sharing")
+DEFAULT_SPLIT = {"continuous_batch": 2048, "large_pool_b16": 2048, "large_pool_b32": 2048,
+                 "worked_example": 128, "prefix_sharing": 1024}
+NSETS = 4           # device input/metadata buffer sets: the host may run this many steps ahead
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default 64; 8 for large_pool)")
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--split", type=int, default=2048, help="tokens per split-K range (0: never split)")
+    ap.add_argument("--workload", default="continuous_batch", choices=WORKLOADS)
+    ap.add_argument("--split", type=int, default=None, help="tokens per split-K range (0: never split)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seqs", type=int, default=24)
-    return ap.parse_args()
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for the CPU baseline")
+    a = ap.parse_args(argv)
+    if a.steps is None:
+        a.steps = 8 if a.workload.startswith("large_pool") else 64
+    if a.split is None:
+        a.split = DEFAULT_SPLIT[a.workload]
+    return a
 
 
 def captured_traffic():
@@ -64,9 +82,9 @@ def captured_traffic():
     return int(gb * 1e9)
 
 
-# ---------------------------------------------------------------------------- schedule
+# ---------------------------------------------------------------------------- schedules
 def simulate(sched, n, steps):
-    """Host-side replay of the schedule: per step the uids, token positions and admissions."""
+    """Continuous batch: per step the uids, token positions, admissions and retirements."""
     lens = np.array(sched.initial, np.int64)
     uids = np.arange(n, dtype=np.int64)
     next_uid, pending = n, []
@@ -78,12 +96,43 @@ def simulate(sched, n, steps):
             lens[slot] = plen
             admitted.append((slot, next_uid, plen))
             next_uid += 1
-        pending = []
-        plan.append(dict(uids=uids.copy(), pos=lens.copy(), admitted=admitted,
-                         retire=list(sched.events[t])))
+        plan.append(dict(uids=uids.copy(), pos=lens.copy(), admitted=admitted, retire=list(sched.events[t])))
         lens += 1
         pending = list(sched.events[t])
     return plan
+
+
+def static_plan(uids, lens, steps):
+    """Fixed batch: every sequence grows by one token per step."""
+    uids = np.asarray(uids, np.int64)
+    lens = np.asarray(lens, np.int64)
+    return [dict(uids=uids.copy(), pos=lens + t, admitted=[], retire=[]) for t in range(steps)]
+
+
+def make_recipe(workload, seed_offset, steps):
+    from synthetic import workloads as wl
+    if workload == "continuous_batch":
+        return wl.continuous_batch(seed=3 + seed_offset, steps=steps)
+    if workload.startswith("large_pool"):
+        return wl.large_pool(seed=5 + seed_offset, block_size=int(workload[-2:]))
+    if workload == "worked_example":
+        return wl.worked_example(seed=2 + seed_offset)
+    return wl.prefix_sharing(seed=4 + seed_offset)
+
+
+def describe(workload):
+    return {
+        "continuous_batch": "continuous_batch: 256 seqs, lengths U[128,4096], block 16, 32 q / 8 KV heads, d128, "
+                            "bf16, p_stop 1/200, 1 layer",
+        "large_pool_b16": "large_pool: 384 seqs, lognormal lengths (median 1500, sigma 0.75, cap 16384), "
+                          "block 16, 32 layers, 32 q / 8 KV heads, d128, fp16, ~100 GB pool",
+        "large_pool_b32": "large_pool: 384 seqs, lognormal lengths (median 1500, sigma 0.75, cap 16384), "
+                          "block 32, 32 layers, 32 q / 8 KV heads, d128, fp16, ~100 GB pool",
+        "worked_example": "worked_example: 4 seqs of 3900/420/2100/70 tokens, block 16, 32 q / 8 KV heads, "
+                          "d128, fp16, 1 layer",
+        "prefix_sharing": "prefix_sharing: 64 seqs sharing a 2048-token prefix + private suffixes U[16,512], "
+                          "block 16, 32 q / 8 KV heads, d128, fp16, 1 layer",
+    }[workload]
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -155,163 +204,215 @@ def combine_ranks(dist, times_ms, byte_counts, device):
 
 
 def replica_seed(rank: int) -> int:
-    """Each rank runs an independent replica of the workload with its own draws."""
-    return 3 + 100 * rank
+    """Seed offset of each rank's replica: every rank draws its own workload."""
+    return 100 * rank
 
 
 # ---------------------------------------------------------------------------- our path
 class Replica:
-    """One GPU's continuous-batch state, inputs pre-generated in HBM."""
+    """One GPU's decode state: pools, block manager, sequences, and every step's inputs
+    generated in HBM before timing starts."""
 
-    def __init__(self, torch, recipe, total_steps, split, device, e2e_from):
+    def __init__(self, torch, workload, recipe, total_steps, split, device, e2e_from):
         from paged_kv_cache_403_b200.engine import PagedCache
         from paged_kv_cache_403_b200.runners import DeviceGen, prefill
         import paged_kv_cache_403_b200 as pa
         self.torch, self.pa = torch, pa
-        self.recipe, self.shape = recipe, recipe["shape"]
+        self.workload, self.recipe, self.shape = workload, recipe, recipe["shape"]
         sh = self.shape
-        self.n = n = len(recipe["schedule"].initial)
-        self.split = split
-        self.device = device
-        self.plan = simulate(recipe["schedule"], n, total_steps)
+        self.NL = sh.num_layers
+        self.split, self.device = split, device
         self.cache = PagedCache.from_shape(sh, recipe["order"], device)
         gen = DeviceGen(recipe["seed"], sh, device)
-        self.sids = [self.cache.add() for _ in range(n)]
-        prefill(self.cache, gen, self.sids, list(range(n)), [int(x) for x in recipe["schedule"].initial])
-        self.max_blocks = -(-(4096 + total_steps + 1) // sh.block_size)
-        # per-step inputs, generated on the device before any timing
-        self.q, self.kn, self.vn, self.pk, self.pv = [], [], [], [], []
-        for t, st in enumerate(self.plan):
-            k, v = gen.kv(0, st["uids"], st["pos"])
-            self.kn.append(k)
-            self.vn.append(v)
-            self.q.append(gen.q(0, st["uids"], st["pos"]))
-            if st["admitted"]:
-                u = np.concatenate([np.full(p, uid) for _, uid, p in st["admitted"]])
-                tk = np.concatenate([np.arange(p) for _, _, p in st["admitted"]])
-                pk, pv = gen.kv(0, u, tk)
-            else:
+        if workload == "continuous_batch":
+            n = len(recipe["schedule"].initial)
+            self.plan = simulate(recipe["schedule"], n, total_steps)
+            self.sids = [self.cache.add() for _ in range(n)]
+            prefill(self.cache, gen, self.sids, list(range(n)), [int(x) for x in recipe["schedule"].initial])
+            self.max_blocks = -(-(4096 + total_steps + 1) // sh.block_size)
+        elif workload == "prefix_sharing":
+            n = len(recipe["suffix"])
+            prefix, suffix = recipe["prefix"], [int(x) for x in recipe["suffix"]]
+            root = self.cache.add()
+            prefill(self.cache, gen, [root], [0], [prefix])
+            self.sids = [root] + [self.cache.fork(root) for _ in range(n - 1)]
+            slots, _ = self.cache.reserve(self.sids, suffix)
+            u = np.repeat(np.arange(n), suffix)
+            tk = np.concatenate([prefix + np.arange(x) for x in suffix])
+            k, v = gen.kv(0, u, tk)
+            self.cache.append(0, k, v, torch.from_numpy(np.ascontiguousarray(slots)).to(device))
+            lens = [prefix + x for x in suffix]
+            self.plan = static_plan(range(n), lens, total_steps)
+            self.max_blocks = -(-(max(lens) + total_steps + 1) // sh.block_size)
+        else:
+            lens = [int(x) for x in recipe["lens"]]
+            n = len(lens)
+            self.sids = [self.cache.add() for _ in range(n)]
+            prefill(self.cache, gen, self.sids, list(range(n)), lens)
+            self.plan = static_plan(range(n), lens, total_steps)
+            self.max_blocks = -(-(max(lens) + total_steps + 1) // sh.block_size)
+        self.n = n
+        # every step's inputs (all layers), generated on the device before any timing
+        self.inputs = []
+        for st in self.plan:
+            per_layer = []
+            for layer in range(self.NL):
+                k, v = gen.kv(layer, st["uids"], st["pos"])
+                q = gen.q(layer, st["uids"], st["pos"])
                 pk = pv = None
-            self.pk.append(pk)
-            self.pv.append(pv)
-        # host copies for the end-to-end variant (pinned)
+                if st["admitted"]:
+                    u = np.concatenate([np.full(p, uid) for _, uid, p in st["admitted"]])
+                    tk = np.concatenate([np.arange(p) for _, _, p in st["admitted"]])
+                    pk, pv = gen.kv(layer, u, tk)
+                per_layer.append((q, k, v, pk, pv))
+            self.inputs.append(per_layer)
+        torch.cuda.synchronize()
         self.host = {}
-        if e2e_from is not None:
+        if e2e_from is not None:      # pinned host copies for the end-to-end leg
             for t in range(e2e_from, total_steps):
-                self.host[t] = [None if x is None else x.cpu().pin_memory()
-                                for x in (self.q[t], self.kn[t], self.vn[t], self.pk[t], self.pv[t])]
-        # metadata: pinned host staging (3 sets) and device buffers (2 sets)
+                self.host[t] = [[None if x is None else x.cpu().pin_memory() for x in lay]
+                                for lay in self.inputs[t]]
         mb = self.max_blocks
         pin = lambda shape, dt: torch.empty(shape, dtype=dt).pin_memory()  # noqa: E731
-        self.h_tables = [pin((n, mb), torch.int32) for _ in range(3)]
-        self.h_lens = [pin((n,), torch.int32) for _ in range(3)]
-        self.h_slots = [pin((n,), torch.int64) for _ in range(3)]
         max_prompt = max([sum(p for _, _, p in st["admitted"]) for st in self.plan] + [1])
-        self.h_pslots = [pin((max_prompt,), torch.int64) for _ in range(3)]
-        self.h_cow = [pin((n, 2), torch.int32) for _ in range(3)]
-        self.h_done = [None, None, None]
-        self.d_tables = [torch.empty((n, mb), dtype=torch.int32, device=device) for _ in range(2)]
-        self.d_lens = [torch.empty((n,), dtype=torch.int32, device=device) for _ in range(2)]
-        self.d_slots = [torch.empty((n,), dtype=torch.int64, device=device) for _ in range(2)]
-        self.d_pslots = [torch.empty((max_prompt,), dtype=torch.int64, device=device) for _ in range(2)]
-        self.d_free = [None, None]
-        self.d_in = [[torch.empty_like(x) for x in (self.q[0], self.kn[0], self.vn[0])] for _ in range(2)]
-        self.d_pk = [torch.empty((max_prompt, sh.num_kv_heads, sh.head_dim), dtype=self.q[0].dtype,
-                                 device=device) for _ in range(2)]
-        self.d_pv = [torch.empty_like(self.d_pk[0]) for _ in range(2)]
-        self.out = torch.empty((n, sh.num_q_heads, sh.head_dim), dtype=self.q[0].dtype, device=device)
-        self.h_out = [pin(tuple(self.out.shape), self.out.dtype) for _ in range(2)]
+        H, D2 = NSETS + 1, NSETS
+        self.h_tables = [pin((n, mb), torch.int32) for _ in range(H)]
+        self.h_lens = [pin((n,), torch.int32) for _ in range(H)]
+        self.h_slots = [pin((n,), torch.int64) for _ in range(H)]
+        self.h_pslots = [pin((max_prompt,), torch.int64) for _ in range(H)]
+        self.h_cow = [pin((n, 2), torch.int32) for _ in range(H)]
+        self.h_done = [None] * H
+        self.d_tables = [torch.empty((n, mb), dtype=torch.int32, device=device) for _ in range(D2)]
+        self.d_lens = [torch.empty((n,), dtype=torch.int32, device=device) for _ in range(D2)]
+        self.d_slots = [torch.empty((n,), dtype=torch.int64, device=device) for _ in range(D2)]
+        self.d_pslots = [torch.empty((max_prompt,), dtype=torch.int64, device=device) for _ in range(D2)]
+        self.d_cow = [torch.empty((n, 2), dtype=torch.int32, device=device) for _ in range(D2)]
+        self.d_free = [None] * D2
+        dt = self.inputs[0][0][0].dtype
+        if e2e_from is not None:
+            self.d_in = [[[torch.empty_like(x) for x in lay[:3]] for lay in self.inputs[0]] for _ in range(D2)]
+            self.d_pk = [[torch.empty((max_prompt, sh.num_kv_heads, sh.head_dim), dtype=dt, device=device)
+                          for _ in range(self.NL)] for _ in range(D2)]
+            self.d_pv = [[torch.empty_like(x) for x in self.d_pk[0]] for _ in range(D2)]
+        self.out = [torch.empty((self.NL, n, sh.num_q_heads, sh.head_dim), dtype=dt, device=device)
+                    for _ in range(D2)]
+        self.h_out = [pin(tuple(self.out[0].shape), dt) for _ in range(D2)] if e2e_from is not None else None
+        self.out_read = [None] * D2
         self.ws = self.cache.workspace(n, sh.num_q_heads, mb, split)
         self.compute = torch.cuda.current_stream(device)
         self.copy = torch.cuda.Stream(device)
+        self.readback = torch.cuda.Stream(device)
         self.scale = 1.0 / math.sqrt(sh.head_dim)
         self.attn_events = []
-        self.kv_bytes = []
-        self.alg_bytes = []
-        self.launches_before = 0
+        self.kv_bytes, self.alg_bytes, self.h2d, self.d2h = [], [], [], []
 
     def step(self, t, e2e=False, time_attention=True):
         torch, pa, sh, plan = self.torch, self.pa, self.shape, self.plan[t]
-        n, hs, ds = self.n, t % 3, t % 2
-        # host staging set hs is free once the copies that used it (3 steps ago) are done
-        if self.h_done[hs] is not None:
+        n, hs, ds = self.n, t % (NSETS + 1), t % NSETS
+        if self.h_done[hs] is not None:      # staging set hs: its uploads (NSETS + 1 steps ago) are done
             self.h_done[hs].synchronize()
-        # 1. admissions: new sequences take the retired slots, their prompts are appended
+        # 1. admissions: new sequences take the retired slots; their prompts are appended below
         ptot = 0
         if plan["admitted"]:
             new = []
             for slot, _, plen in plan["admitted"]:
                 self.sids[slot] = self.cache.add()
                 new.append((self.sids[slot], plen))
-            pslots, cow = pa.pa_reserve_slots(self.cache.pool, [s for s, _ in new], [p for _, p in new],
-                                              slot_out=self.h_pslots[hs])
+            pslots, _ = pa.pa_reserve_slots(self.cache.pool, [s for s, _ in new], [p for _, p in new],
+                                            slot_out=self.h_pslots[hs])
             ptot = len(pslots)
-        # 2. one slot per sequence for this step's token (new block or copy-on-write)
-        slots, cow = pa.pa_reserve_slots(self.cache.pool, self.sids, [1] * n, slot_out=self.h_slots[hs],
-                                         cow_out=self.h_cow[hs])
-        assert len(cow) == 0          # no sharing in this workload
-        tables, lens = pa.pa_build_block_tables(self.cache.pool, self.sids, self.max_blocks,
-                                                self.h_tables[hs], self.h_lens[hs])
-        # 3. upload metadata (and, end to end, the step's inputs) on the copy stream
+        # 2. one slot per sequence for this step's token (new block, or copy-on-write of a shared tail)
+        _, cow = pa.pa_reserve_slots(self.cache.pool, self.sids, [1] * n, slot_out=self.h_slots[hs],
+                                     cow_out=self.h_cow[hs])
+        ncow = len(cow)
+        _, lens = pa.pa_build_block_tables(self.cache.pool, self.sids, self.max_blocks, self.h_tables[hs],
+                                           self.h_lens[hs])
+        # 3. uploads (metadata; end to end also the step's inputs) on the copy stream
         if self.d_free[ds] is not None:
             self.copy.wait_event(self.d_free[ds])
+        h2d = self.h_tables[hs].numel() * 4 + n * 4 + n * 8 + ptot * 8 + ncow * 8
         with torch.cuda.stream(self.copy):
             self.d_tables[ds].copy_(self.h_tables[hs], non_blocking=True)
             self.d_lens[ds].copy_(self.h_lens[hs], non_blocking=True)
             self.d_slots[ds].copy_(self.h_slots[hs], non_blocking=True)
             if ptot:
                 self.d_pslots[ds][:ptot].copy_(self.h_pslots[hs][:ptot], non_blocking=True)
+            if ncow:
+                self.d_cow[ds][:ncow].copy_(self.h_cow[hs][:ncow], non_blocking=True)
             if e2e:
-                hq, hk, hv, hpk, hpv = self.host[t]
-                q, kn, vn = self.d_in[ds]
-                q.copy_(hq, non_blocking=True)
-                kn.copy_(hk, non_blocking=True)
-                vn.copy_(hv, non_blocking=True)
-                if ptot:
-                    self.d_pk[ds][:ptot].copy_(hpk, non_blocking=True)
-                    self.d_pv[ds][:ptot].copy_(hpv, non_blocking=True)
-                pk, pv = self.d_pk[ds][:ptot], self.d_pv[ds][:ptot]
+                layers = []
+                for layer, host in enumerate(self.host[t]):
+                    q, k, v = self.d_in[ds][layer]
+                    for dst, src in ((q, host[0]), (k, host[1]), (v, host[2])):
+                        dst.copy_(src, non_blocking=True)
+                        h2d += src.numel() * src.element_size()
+                    pk = pv = None
+                    if ptot:
+                        pk, pv = self.d_pk[ds][layer][:ptot], self.d_pv[ds][layer][:ptot]
+                        pk.copy_(host[3], non_blocking=True)
+                        pv.copy_(host[4], non_blocking=True)
+                        h2d += 2 * host[3].numel() * host[3].element_size()
+                    layers.append((q, k, v, pk, pv))
             else:
-                q, kn, vn, pk, pv = self.q[t], self.kn[t], self.vn[t], self.pk[t], self.pv[t]
+                layers = self.inputs[t]
             up = torch.cuda.Event()
             up.record(self.copy)
         self.h_done[hs] = up
         self.compute.wait_event(up)
-        # 4. device work on the compute stream
-        if ptot:
-            pa.pa_append_kv(self.cache.pool, 0, pk, pv, self.d_pslots[ds], ptot, stream=self.compute)
-        pa.pa_append_kv(self.cache.pool, 0, kn, vn, self.d_slots[ds], n, stream=self.compute)
-        if time_attention:
-            e0 = torch.cuda.Event(enable_timing=True)
-            e0.record(self.compute)
-        pa.pa_decode_attention(self.cache.pool, 0, q, self.out, self.d_tables[ds], self.d_lens[ds], self.scale,
-                               self.split, self.ws, stream=self.compute)
-        if time_attention:
-            e1 = torch.cuda.Event(enable_timing=True)
-            e1.record(self.compute)
-            self.attn_events.append((e0, e1))
+        if self.out_read[ds] is not None:    # the read-back of out[ds] (NSETS steps ago) is done
+            self.compute.wait_event(self.out_read[ds])
+        # 4. device work
+        if ncow:
+            pa.pa_copy_blocks(self.cache.pool, self.d_cow[ds], ncow, stream=self.compute)
+        for layer, (q, k, v, pk, pv) in enumerate(layers):
+            if ptot:
+                pa.pa_append_kv(self.cache.pool, layer, pk, pv, self.d_pslots[ds], ptot, stream=self.compute)
+            pa.pa_append_kv(self.cache.pool, layer, k, v, self.d_slots[ds], n, stream=self.compute)
+            if time_attention:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e0.record(self.compute)
+            pa.pa_decode_attention(self.cache.pool, layer, q, self.out[ds][layer], self.d_tables[ds],
+                                   self.d_lens[ds], self.scale, self.split, self.ws, stream=self.compute)
+            if time_attention:
+                e1 = torch.cuda.Event(enable_timing=True)
+                e1.record(self.compute)
+                self.attn_events.append((e0, e1))
         free = torch.cuda.Event()
         free.record(self.compute)
         self.d_free[ds] = free
-        if e2e:
-            self.h_out[ds].copy_(self.out, non_blocking=True)
+        d2h = 0
+        if e2e:                              # result read back on its own stream
+            self.readback.wait_event(free)
+            with torch.cuda.stream(self.readback):
+                self.h_out[ds].copy_(self.out[ds], non_blocking=True)
+                rd = torch.cuda.Event()
+                rd.record(self.readback)
+            self.out_read[ds] = rd
+            d2h = self.out[ds].numel() * self.out[ds].element_size()
         # 5. retirements: blocks go back to the free list at once
         for slot, _ in plan["retire"]:
             self.cache.free(self.sids[slot])
-        # accounting (host): KV bytes the attention reads this step
+        # accounting: bytes decode attention reads / writes this step (all layers)
         L = lens.numpy().astype(np.int64)
         e = 2
-        kv = int((2 * L * sh.num_kv_heads * sh.head_dim * e).sum())
-        alg = kv + 2 * n * sh.num_q_heads * sh.head_dim * e + int((4 * -(-L // sh.block_size)).sum()) + 4 * n
+        kv = self.NL * int((2 * L * sh.num_kv_heads * sh.head_dim * e).sum())
+        alg = kv + self.NL * (2 * n * sh.num_q_heads * sh.head_dim * e + int((4 * -(-L // sh.block_size)).sum())
+                              + 4 * n)
         self.kv_bytes.append(kv)
         self.alg_bytes.append(alg)
-        return ptot
+        self.h2d.append(h2d)
+        self.d2h.append(d2h)
+
+    def drain(self):
+        """Make the compute stream wait for outstanding read-backs (end of a timed leg)."""
+        for ev in self.out_read:
+            if ev is not None:
+                self.compute.wait_event(ev)
 
 
 def run_ours(args):
     import torch
     import torch.distributed as dist
-    from synthetic import workloads as wl
     import paged_kv_cache_403_b200 as pa
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -328,9 +429,8 @@ def run_ours(args):
     K, W = args.steps, args.warmup
     e2e = not args.no_e2e
     total = W + K + (K if e2e else 0)
-    recipe = wl.continuous_batch(seed=replica_seed(rank), steps=total)
-    rep = Replica(torch, recipe, total, args.split, device, W + K if e2e else None)
-    torch.cuda.synchronize()
+    recipe = make_recipe(args.workload, replica_seed(rank), total)
+    rep = Replica(torch, args.workload, recipe, total, args.split, device, W + K if e2e else None)
 
     def barrier():
         if world > 1:
@@ -356,81 +456,71 @@ def run_ours(args):
     ms = ev0.elapsed_time(ev1)
     kv_bytes = sum(rep.kv_bytes)
     attn_ms = [a.elapsed_time(b) for a, b in rep.attn_events]
-    alg_bytes = list(rep.alg_bytes)
+    alg_per_launch = sum(rep.alg_bytes) / (K * rep.NL)
 
-    e2e_res = None
+    e2e_ms = e2e_kv = 0.0
+    e2e_io = (0, 0)
     if e2e:
         rep.kv_bytes.clear()
-        rep.alg_bytes.clear()
+        rep.h2d.clear()
+        rep.d2h.clear()
         barrier()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(rep.compute)
-        h2d = d2h = 0
         for t in range(W + K, W + 2 * K):
-            ptot = rep.step(t, e2e=True, time_attention=False)
-            sh = rep.shape
-            h2d += (rep.q[t].numel() + rep.kn[t].numel() + rep.vn[t].numel() + 2 * ptot * sh.num_kv_heads
-                    * sh.head_dim) * 2
-            h2d += rep.n * rep.max_blocks * 4 + rep.n * 4 + rep.n * 8 + ptot * 8
-            d2h += rep.out.numel() * 2
+            rep.step(t, e2e=True, time_attention=False)
+        rep.drain()
         t1.record(rep.compute)
         barrier()
-        e_ms = t0.elapsed_time(t1)
-        e_kv = sum(rep.kv_bytes)
-        e2e_res = (e_ms, e_kv, h2d / K, d2h / K)
+        e2e_ms, e2e_kv = t0.elapsed_time(t1), sum(rep.kv_bytes)
+        e2e_io = (sum(rep.h2d) / K, sum(rep.d2h) / K)
     clk = clocks.stop()
 
-    # whole-job numbers: bytes summed over ranks, time = max over ranks
     if world > 1:
-        (ms, e2e_ms), (kv_tot, e2e_kv) = combine_ranks(
-            dist, [ms, e2e_res[0] if e2e_res else 0.0], [kv_bytes, e2e_res[1] if e2e_res else 0], device)
+        (ms, e2e_ms), (kv_tot, e2e_kv) = combine_ranks(dist, [ms, e2e_ms], [kv_bytes, e2e_kv], device)
     else:
         kv_tot = kv_bytes
-        e2e_ms, e2e_kv = (e2e_res[0], e2e_res[1]) if e2e_res else (0.0, 0)
 
     if rank == 0:
-        import json as _json
         peaks = {}
         pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
         if os.path.exists(pk_path):
-            peaks = _json.load(open(pk_path))
+            peaks = json.load(open(pk_path))
         peak = float(peaks.get("hbm_gbs", 6650.0))
         peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
         attn_mean_ms = float(np.mean(attn_ms))
-        alg_mean = float(np.mean(alg_bytes))
-        achieved = alg_mean / (attn_mean_ms * 1e-3) / 1e9
+        achieved = alg_per_launch / (attn_mean_ms * 1e-3) / 1e9
         value = kv_tot / (ms * 1e-3) / 1e9
-        tokens_per_s = world * rep.n * K / (ms * 1e-3)
+        sh = rep.shape
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based K/V/q, "
-            "seeded lengths and stops)",
-            "config": {"workload": "continuous_batch: 256 seqs, lengths U[128,4096], block 16, "
-                       "32 q / 8 KV heads, d128, bf16, p_stop 1/200, 1 layer", "n_seqs": rep.n,
-                       "block_size": 16, "num_q_heads": 32, "num_kv_heads": 8, "head_dim": 128,
-                       "split_tokens": args.split, "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (KV read per step ~2.2 GB > 126 MB)"},
-            "decode_tokens_per_s": round(tokens_per_s, 1),
+            "vs_baseline": None, "dtype": sh.dtype,
+            "data": "synthetic (seeded counter-based K/V/q values; seeded lengths, pool order and stops)",
+            "config": {"workload": describe(args.workload), "n_seqs": rep.n, "num_layers": rep.NL,
+                       "block_size": sh.block_size, "num_q_heads": sh.num_q_heads,
+                       "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim, "split_tokens": args.split,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "no flush: the KV read per step exceeds the 126 MB L2"},
+            "decode_tokens_per_s": round(world * rep.n * K / (ms * 1e-3), 1),
             "kv_gb_per_step": round(kv_tot / K / 1e9 / world, 4),
             "hbm_fraction_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": captured_traffic(),
+                         "frac": round(achieved / peak, 4),
+                         "traffic": captured_traffic() if args.workload == "continuous_batch" else None,
                          "kernel": "paged_decode_mma_kernel (+ split_reduce_kernel)",
-                         "attn_ms_mean": round(attn_mean_ms, 4),
-                         "alg_bytes_per_launch": int(alg_mean), "peak_source": peak_src},
+                         "attn_ms_mean": round(attn_mean_ms, 4), "alg_bytes_per_launch": int(alg_per_launch),
+                         "launches_timed": len(attn_ms), "peak_source": peak_src},
             "gpu_launches": int(launches),
             "clocks": clk,
         }
-        if e2e_res:
+        if e2e:
             line["e2e"] = {"value": round(e2e_kv / (e2e_ms * 1e-3) / 1e9, 1), "unit": UNIT,
-                           "h2d_bytes_per_step": int(e2e_res[2]), "d2h_bytes_per_step": int(e2e_res[3]),
+                           "h2d_bytes_per_step": int(e2e_io[0]), "d2h_bytes_per_step": int(e2e_io[1]),
                            "ms_per_step": round(e2e_ms / K, 4)}
-        if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(recipe, rep, args.cpu_sample_seqs, W)
-        elif not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(recipe, rep, args.cpu_sample_seqs, W)
+        if not args.no_cpu_baseline and args.workload != "prefix_sharing":
+            line["cpu_baseline"] = cpu_baseline(rep, args.cpu_sample_seqs, W, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -438,8 +528,9 @@ def run_ours(args):
 
 
 # ---------------------------------------------------------------------------- oracle (CPU)
-def oracle_sample(recipe, plan_step, picks):
-    """Host inputs (regenerated) for the sampled sequences of one step: contiguous pools."""
+def oracle_sample(recipe, plan_step, picks, layer=0):
+    """Host inputs for the sampled sequences of one step, regenerated from the seeded
+    generator (never read from the GPU): each sequence's history laid contiguously."""
     from synthetic import values as sv
     sh = recipe["shape"]
     B, hkv, d = sh.block_size, sh.num_kv_heads, sh.head_dim
@@ -448,8 +539,8 @@ def oracle_sample(recipe, plan_step, picks):
     for i in picks:
         uid, L = int(plan_step["uids"][i]), int(plan_step["pos"][i]) + 1
         pos = np.arange(L)
-        k = sv.rows(sv.KIND_K, recipe["seed"], 0, np.full(L, uid), pos, hkv, d, sh.kv_scale, sh.dtype)
-        v = sv.rows(sv.KIND_V, recipe["seed"], 0, np.full(L, uid), pos, hkv, d, sh.kv_scale, sh.dtype)
+        k = sv.rows(sv.KIND_K, recipe["seed"], layer, np.full(L, uid), pos, hkv, d, sh.kv_scale, sh.dtype)
+        v = sv.rows(sv.KIND_V, recipe["seed"], layer, np.full(L, uid), pos, hkv, d, sh.kv_scale, sh.dtype)
         nblk = -(-L // B)
         pad = nblk * B - L
         k = np.concatenate([k, np.zeros((pad, hkv, d), k.dtype)]).reshape(nblk, B, hkv, d).transpose(0, 2, 1, 3)
@@ -459,7 +550,7 @@ def oracle_sample(recipe, plan_step, picks):
         tabs.append(np.arange(nb, nb + nblk))
         nb += nblk
         lens.append(L)
-        qs.append(sv.rows(sv.KIND_Q, recipe["seed"], 0, [uid], [L - 1], sh.num_q_heads, d, sh.q_scale,
+        qs.append(sv.rows(sv.KIND_Q, recipe["seed"], layer, [uid], [L - 1], sh.num_q_heads, d, sh.q_scale,
                           sh.dtype)[0])
     mb = max(len(t) for t in tabs)
     tables = np.full((len(picks), mb), -1, np.int32)
@@ -469,24 +560,30 @@ def oracle_sample(recipe, plan_step, picks):
             np.array(lens, np.int32), np.stack(qs))
 
 
-def time_oracle(recipe, plan_step, picks):
+def time_oracle(recipe, plan_step, picks, min_seconds=0.0, max_reps=1000):
+    """Runs the oracle (as it stands) on the sample, repeated until min_seconds have passed."""
     import oracle
     sh = recipe["shape"]
     k, v, tables, lens, q = oracle_sample(recipe, plan_step, picks)
-    t0 = time.perf_counter()
-    oracle.paged_decode(k, v, sh.dtype, tables, lens, q, 1.0 / math.sqrt(sh.head_dim))
-    dt = time.perf_counter() - t0
-    kv = int((2 * lens.astype(np.int64) * sh.num_kv_heads * sh.head_dim * 2).sum())
-    return kv, dt
+    kv1 = int((2 * lens.astype(np.int64) * sh.num_kv_heads * sh.head_dim * 2).sum())
+    reps, dt = 0, 0.0
+    while reps < max_reps and (reps == 0 or dt < min_seconds):
+        t0 = time.perf_counter()
+        oracle.paged_decode(k, v, sh.dtype, tables, lens, q, 1.0 / math.sqrt(sh.head_dim))
+        dt += time.perf_counter() - t0
+        reps += 1
+    return kv1 * reps, dt, reps, kv1
 
 
-def cpu_baseline(recipe, rep, nseq, step):
+def cpu_baseline(rep, nseq, step, seconds):
     import oracle
     picks = list(range(0, rep.n, max(1, rep.n // nseq)))[:nseq]
-    kv, dt = time_oracle(recipe, rep.plan[step], picks)
+    kv, dt, reps, kv1 = time_oracle(rep.recipe, rep.plan[step], picks, min_seconds=seconds)
+    layers = f"; 1 of {rep.NL} layers" if rep.NL > 1 else ""
     return {"value": round(kv / dt / 1e9, 4), "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
             "sample": f"fp64 oracle attention for {len(picks)} of {rep.n} sequences of one decode step "
-                      f"({kv / 1e6:.1f} MB of KV), OpenMP over (sequence, head)", "seconds": round(dt, 3)}
+                      f"({kv1 / 1e6:.1f} MB of KV{layers}), repeated {reps}x for {dt:.1f} s; "
+                      "OpenMP over (sequence, head)"}
 
 
 def run_reference(args):
@@ -504,17 +601,16 @@ def run_reference(args):
         time_oracle(recipe, plan[t], list(range(t * nseq % 256, t * nseq % 256 + nseq)))
     kv_tot, dt_tot = 0, 0.0
     for t in range(W, W + K):
-        kv, dt = time_oracle(recipe, plan[t], list(range(t * nseq % 256, t * nseq % 256 + nseq)))
+        kv, dt, _, _ = time_oracle(recipe, plan[t], list(range(t * nseq % 256, t * nseq % 256 + nseq)))
         kv_tot += kv
         dt_tot += dt
     value = kv_tot / dt_tot / 1e9
-    sample = (f"each step: fp64 oracle attention for {nseq} of 256 sequences (KV bytes of those "
-              f"sequences / oracle wall time), OpenMP over (sequence, head)")
+    sample = (f"each step: fp64 oracle attention for {nseq} of the 256 sequences of that step (KV bytes of "
+              "those sequences / oracle wall time), OpenMP over (sequence, head)")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": round(dt_tot / K * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "continuous_batch: 256 seqs, lengths U[128,4096], block 16, 32 q / 8 KV "
-                       "heads, d128, bf16, p_stop 1/200, 1 layer", "parallelism": "cpu"},
+            "config": {"workload": describe("continuous_batch"), "parallelism": "cpu"},
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oracle.max_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
