@@ -38,9 +38,10 @@ sys.path.insert(0, ROOT)
 METRIC = "paged decode attention KV-read HBM GB/s (fraction of ~8 TB/s) and decode tokens/s"
 UNIT = "GB/s"
 NOMINAL_HBM_GBS = 8000.0
-WORKLOADS = ("continuous_batch", "large_pool_b16", "large_pool_b32", "worked_example", "prefix_sharing")
+WORKLOADS = ("continuous_batch", "large_pool_b16", "large_pool_b32", "worked_example", "prefix_sharing",
+             "shared_prompt")
 DEFAULT_SPLIT = {"continuous_batch": 2048, "large_pool_b16": 2048, "large_pool_b32": 2048,
-                 "worked_example": 128, "prefix_sharing": 1024}
+                 "worked_example": 128, "prefix_sharing": 1024, "shared_prompt": 2048}
 NSETS = 4           # device input/metadata buffer sets: the host may run this many steps ahead
 
 
@@ -56,6 +57,8 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seqs", type=int, default=24)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for the CPU baseline")
+    ap.add_argument("--prefix-cache", default="on", choices=["on", "off"],
+                    help="shared_prompt workload: share the cached system-prompt blocks at admission")
     a = ap.parse_args(argv)
     if a.steps is None:
         a.steps = 8 if a.workload.startswith("large_pool") else 64
@@ -117,6 +120,8 @@ def make_recipe(workload, seed_offset, steps):
         return wl.large_pool(seed=5 + seed_offset, block_size=int(workload[-2:]))
     if workload == "worked_example":
         return wl.worked_example(seed=2 + seed_offset)
+    if workload == "shared_prompt":
+        return wl.shared_prompt_batch(seed=6 + seed_offset, steps=steps)
     return wl.prefix_sharing(seed=4 + seed_offset)
 
 
@@ -132,6 +137,9 @@ def describe(workload):
                           "d128, fp16, 1 layer",
         "prefix_sharing": "prefix_sharing: 64 seqs sharing a 2048-token prefix + private suffixes U[16,512], "
                           "block 16, 32 q / 8 KV heads, d128, fp16, 1 layer",
+        "shared_prompt": "shared_prompt: continuous batch of 256 seqs whose prompts (U[1152,4096] tokens) start "
+                         "with one 1024-token system prompt, block 16, 32 q / 8 KV heads, d128, bf16, "
+                         "p_stop 1/200, 1 layer",
     }[workload]
 
 
@@ -213,7 +221,7 @@ class Replica:
     """One GPU's decode state: pools, block manager, sequences, and every step's inputs
     generated in HBM before timing starts."""
 
-    def __init__(self, torch, workload, recipe, total_steps, split, device, e2e_from):
+    def __init__(self, torch, workload, recipe, total_steps, split, device, e2e_from, prefix_cache=True):
         from paged_kv_cache_403_b200.engine import PagedCache
         from paged_kv_cache_403_b200.runners import DeviceGen, prefill
         import paged_kv_cache_403_b200 as pa
@@ -224,12 +232,27 @@ class Replica:
         self.split, self.device = split, device
         self.cache = PagedCache.from_shape(sh, recipe["order"], device)
         gen = DeviceGen(recipe["seed"], sh, device)
+        self.prompt_start = lambda plen: 0          # first prompt position an admission appends
+        self.system_keys = None
         if workload == "continuous_batch":
             n = len(recipe["schedule"].initial)
             self.plan = simulate(recipe["schedule"], n, total_steps)
             self.sids = [self.cache.add() for _ in range(n)]
             prefill(self.cache, gen, self.sids, list(range(n)), [int(x) for x in recipe["schedule"].initial])
             self.max_blocks = -(-(4096 + total_steps + 1) // sh.block_size)
+        elif workload == "shared_prompt":
+            from paged_kv_cache_403_b200.runners import SharedPromptBatch
+            n = len(recipe["schedule"].initial)
+            self.max_blocks = -(-(4096 + total_steps + 1) // sh.block_size)
+            sb = SharedPromptBatch(recipe, device, self.max_blocks, cache=prefix_cache)
+            self.cache.close()
+            self.cache, self.sids = sb.cache, sb.sids
+            self.plan = simulate(recipe["schedule"], n, total_steps)
+            if prefix_cache:
+                self.system_keys = sb.keys
+                self.prompt_start = lambda plen: recipe["system"]
+            self.prompt_rows = lambda uid, plen: sb._rows(uid, plen, recipe["system"], recipe["system_uid"],
+                                                          self.prompt_start(plen))
         elif workload == "prefix_sharing":
             n = len(recipe["suffix"])
             prefix, suffix = recipe["prefix"], [int(x) for x in recipe["suffix"]]
@@ -261,8 +284,11 @@ class Replica:
                 q = gen.q(layer, st["uids"], st["pos"])
                 pk = pv = None
                 if st["admitted"]:
-                    u = np.concatenate([np.full(p, uid) for _, uid, p in st["admitted"]])
-                    tk = np.concatenate([np.arange(p) for _, _, p in st["admitted"]])
+                    if workload == "shared_prompt":
+                        u, tk = map(np.concatenate, zip(*[self.prompt_rows(uid, p) for _, uid, p in st["admitted"]]))
+                    else:
+                        u = np.concatenate([np.full(p, uid) for _, uid, p in st["admitted"]])
+                        tk = np.concatenate([np.arange(p) for _, _, p in st["admitted"]])
                     pk, pv = gen.kv(layer, u, tk)
                 per_layer.append((q, k, v, pk, pv))
             self.inputs.append(per_layer)
@@ -274,7 +300,7 @@ class Replica:
                                 for lay in self.inputs[t]]
         mb = self.max_blocks
         pin = lambda shape, dt: torch.empty(shape, dtype=dt).pin_memory()  # noqa: E731
-        max_prompt = max([sum(p for _, _, p in st["admitted"]) for st in self.plan] + [1])
+        max_prompt = max([sum(p - self.prompt_start(p) for _, _, p in st["admitted"]) for st in self.plan] + [1])
         H, D2 = NSETS + 1, NSETS
         self.h_tables = [pin((n, mb), torch.int32) for _ in range(H)]
         self.h_lens = [pin((n,), torch.int32) for _ in range(H)]
@@ -304,7 +330,7 @@ class Replica:
         self.readback = torch.cuda.Stream(device)
         self.scale = 1.0 / math.sqrt(sh.head_dim)
         self.attn_events = []
-        self.kv_bytes, self.alg_bytes, self.h2d, self.d2h = [], [], [], []
+        self.kv_bytes, self.alg_bytes, self.h2d, self.d2h, self.prompt_rows_appended = [], [], [], [], []
 
     def step(self, t, e2e=False, time_attention=True):
         torch, pa, sh, plan = self.torch, self.pa, self.shape, self.plan[t]
@@ -316,11 +342,17 @@ class Replica:
         if plan["admitted"]:
             new = []
             for slot, _, plen in plan["admitted"]:
-                self.sids[slot] = self.cache.add()
-                new.append((self.sids[slot], plen))
+                if self.system_keys is not None:       # share the cached system-prompt blocks
+                    sid, hit = pa.pa_seq_add_cached(self.cache.pool, self.system_keys)
+                    assert hit * sh.block_size == self.prompt_start(plen)
+                else:
+                    sid = self.cache.add()
+                self.sids[slot] = sid
+                new.append((sid, plen - self.prompt_start(plen)))
             pslots, _ = pa.pa_reserve_slots(self.cache.pool, [s for s, _ in new], [p for _, p in new],
                                             slot_out=self.h_pslots[hs])
             ptot = len(pslots)
+        self.prompt_rows_appended.append(ptot)
         # 2. one slot per sequence for this step's token (new block, or copy-on-write of a shared tail)
         _, cow = pa.pa_reserve_slots(self.cache.pool, self.sids, [1] * n, slot_out=self.h_slots[hs],
                                      cow_out=self.h_cow[hs])
@@ -430,7 +462,8 @@ def run_ours(args):
     e2e = not args.no_e2e
     total = W + K + (K if e2e else 0)
     recipe = make_recipe(args.workload, replica_seed(rank), total)
-    rep = Replica(torch, args.workload, recipe, total, args.split, device, W + K if e2e else None)
+    rep = Replica(torch, args.workload, recipe, total, args.split, device, W + K if e2e else None,
+                  prefix_cache=args.prefix_cache == "on")
 
     def barrier():
         if world > 1:
@@ -441,6 +474,7 @@ def run_ours(args):
         rep.step(t, time_attention=False)
     rep.kv_bytes.clear()
     rep.alg_bytes.clear()
+    rep.prompt_rows_appended.clear()
     barrier()
     clocks = ClockSampler(local)
     clocks.start()
@@ -455,6 +489,7 @@ def run_ours(args):
     launches = pa.pa_launch_count() - lc0
     ms = ev0.elapsed_time(ev1)
     kv_bytes = sum(rep.kv_bytes)
+    prompt_rows = sum(rep.prompt_rows_appended)
     attn_ms = [a.elapsed_time(b) for a, b in rep.attn_events]
     alg_per_launch = sum(rep.alg_bytes) / (K * rep.NL)
 
@@ -515,11 +550,19 @@ def run_ours(args):
             "gpu_launches": int(launches),
             "clocks": clk,
         }
+        stats = rep.pa.pa_pool_stats(rep.cache.pool)
+        line["pool"] = {"peak_blocks_used": stats["peak_used"], "num_blocks": stats["num_blocks"],
+                        "cache_hits": stats["cache_hits"], "cached_blocks": stats["num_cached"],
+                        "prompt_rows_appended_per_step": round(prompt_rows / K, 1),
+                        "prompt_bytes_appended_per_step": int(prompt_rows / K * 2 * sh.num_kv_heads
+                                                              * sh.head_dim * 2 * rep.NL)}
+        if args.workload == "shared_prompt":
+            line["config"]["prefix_cache"] = args.prefix_cache
         if e2e:
             line["e2e"] = {"value": round(e2e_kv / (e2e_ms * 1e-3) / 1e9, 1), "unit": UNIT,
                            "h2d_bytes_per_step": int(e2e_io[0]), "d2h_bytes_per_step": int(e2e_io[1]),
                            "ms_per_step": round(e2e_ms / K, 4)}
-        if not args.no_cpu_baseline and args.workload != "prefix_sharing":
+        if not args.no_cpu_baseline and args.workload not in ("prefix_sharing", "shared_prompt"):
             line["cpu_baseline"] = cpu_baseline(rep, args.cpu_sample_seqs, W, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -75,6 +75,10 @@ typedef struct {
     int64_t num_tokens;        /* sum of live sequence lengths */
     int64_t cow_copies;        /* copy-on-write pairs issued so far */
     int32_t peak_used;         /* most blocks ever in use at once */
+    int32_t num_cached;        /* blocks registered for prefix caching */
+    int32_t num_evictable;     /* registered blocks with refcount 0 (counted in num_free) */
+    int64_t cache_hits;        /* blocks shared through pa_seq_add_cached */
+    int64_t cache_evictions;   /* registered blocks reclaimed by allocation */
 } pa_pool_stats_t;
 
 /* Message for the last failing call on this thread ("" if none). */
@@ -153,6 +157,37 @@ pa_status pa_reserve_slots(pa_pool *pool, const int32_t *seq_ids, const int32_t 
  * PA_ERR_INVALID_ARG if a sequence has more than max_blocks blocks. */
 pa_status pa_build_block_tables(const pa_pool *pool, const int32_t *seq_ids, int32_t n,
                                 int32_t max_blocks, int32_t *tables_out, int32_t *lens_out);
+
+/* ------------------------------------------------------------------ prefix caching */
+
+/* [P1] "How PagedAttention works": prefix caching can reuse blocks the way shared
+ * beams do; [P2] "If you remember three things": shared prefixes are shared
+ * blocks.  The pages define no lookup, so the key of a full block is the caller's:
+ * typically a hash chain over the block's token ids and every token before it, so
+ * equal keys mean equal key/value contents.
+ *  - A registered block keeps its key while it lives.  When its refcount reaches 0
+ *    it is not pushed on the free stack: it joins the back of an evictable queue
+ *    and can still be found.  Allocation uses the free stack first and only then
+ *    evicts the front of the queue (least recently released), forgetting its key.
+ *  - pa_num_free_blocks counts free and evictable blocks; pa_free_list lists the
+ *    free stack only, pa_prefix_evictable the queue. */
+
+/* Register the first n_blocks blocks of seq_id (they must be full:
+ * n_blocks * block_size <= length) under keys[0..n_blocks).  A key that is already
+ * registered, or a block that already has a key, is skipped.  *n_new (may be NULL)
+ * receives how many blocks were registered. */
+pa_status pa_prefix_register(pa_pool *pool, int32_t seq_id, const uint64_t *keys, int32_t n_blocks,
+                             int32_t *n_new);
+/* New sequence whose leading blocks are the registered blocks of keys[0..n_keys),
+ * shared (refcount + 1; an evictable block leaves the queue) up to the first key
+ * that is not registered.  *n_hit receives the number shared; the sequence's length
+ * is n_hit * block_size, and the caller appends the rest of its prompt with
+ * pa_reserve_slots / pa_append_kv as usual. */
+pa_status pa_seq_add_cached(pa_pool *pool, const uint64_t *keys, int32_t n_keys, int32_t *seq_id,
+                            int32_t *n_hit);
+/* Copy the evictable queue, front (next to be evicted) first, into out[0..cap);
+ * *n receives its length. */
+pa_status pa_prefix_evictable(const pa_pool *pool, int32_t *out, int32_t cap, int32_t *n);
 
 /* ------------------------------------------------------------------ device work */
 

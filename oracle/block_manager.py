@@ -37,10 +37,28 @@ Readings where the pages leave a step open (each listed in the design notes):
    part way, the whole call fails and nothing changes.
 6. retiring a sequence decrements its blocks in logical order; forking one
    increments its blocks in logical order.
+
+Prefix caching (page 1, same section: "Prefix caching can use a similar idea";
+page 2, "If you remember three things": shared prefixes are shared blocks).  The
+pages give no lookup, so the reading taken is:
+
+7. a full block can be registered under a caller-supplied 64-bit key (a hash
+   chain of its tokens and all tokens before it); a key maps to one block and a
+   block has at most one key; registering an existing key or a registered block
+   changes nothing.
+8. a registered block whose count drops to zero is not pushed on the free
+   stack: it joins the back of an evictable queue (least recently released at
+   the front) and keeps its key.
+9. alloc takes the top of the free stack; only when the stack is empty does it
+   evict the front of the queue (the key is forgotten) and hand that block out.
+10. a new sequence built from keys walks them in order and shares each
+   registered block (count + 1, leaving the queue if it was there) until the
+   first miss; its length is then (hits x B).
 """
 from __future__ import annotations
 
 import copy
+from collections import OrderedDict
 
 
 class OutOfBlocks(Exception):
@@ -69,15 +87,22 @@ class BlockManagerModel:
         self.tables: dict[int, list[int]] = {}
         self.lengths: dict[int, int] = {}
         self.next_seq = 0
+        self.key_of: dict[int, int] = {}            # block -> key (registered blocks)
+        self.block_of: dict[int, int] = {}          # key -> block
+        self.evictable: OrderedDict = OrderedDict()  # registered blocks with count 0, oldest first
 
     # ---- blocks --------------------------------------------------------------
     def num_free(self) -> int:
-        return len(self.free_stack)
+        return len(self.free_stack) + len(self.evictable)
 
     def alloc(self) -> int:
-        if not self.free_stack:
+        if self.free_stack:
+            b = self.free_stack.pop()
+        elif self.evictable:
+            b, _ = self.evictable.popitem(last=False)
+            del self.block_of[self.key_of.pop(b)]
+        else:
             raise OutOfBlocks()
-        b = self.free_stack.pop()
         self.refcount[b] = 1
         return b
 
@@ -87,7 +112,10 @@ class BlockManagerModel:
             raise DoubleFree(b)
         self.refcount[b] -= 1
         if self.refcount[b] == 0:
-            self.free_stack.append(b)
+            if b in self.key_of:
+                self.evictable[b] = None
+            else:
+                self.free_stack.append(b)
 
     def incref(self, b: int) -> None:
         self._check_block(b)
@@ -154,16 +182,51 @@ class BlockManagerModel:
         for s, n in zip(seq_ids, ntok):
             if s not in self.tables or n < 0:
                 raise InvalidArgument(s)
-        saved = copy.deepcopy((self.free_stack, self.refcount, self.tables, self.lengths))
+        saved = copy.deepcopy((self.free_stack, self.refcount, self.tables, self.lengths, self.key_of,
+                               self.block_of, self.evictable))
         slots, cow = [], []
         try:
             for s, n in zip(seq_ids, ntok):
                 for _ in range(n):
                     slots.append(self._append_one(s, cow))
         except OutOfBlocks:
-            self.free_stack, self.refcount, self.tables, self.lengths = saved
+            (self.free_stack, self.refcount, self.tables, self.lengths, self.key_of, self.block_of,
+             self.evictable) = saved
             raise
         return slots, cow
+
+    # ---- prefix caching --------------------------------------------------------
+    def register(self, sid: int, keys) -> int:
+        """Register the first len(keys) blocks of sid (all full) under keys; returns
+        how many were newly registered."""
+        if sid not in self.tables:
+            raise InvalidArgument(sid)
+        keys = [int(k) for k in keys]
+        if len(keys) * self.block_size > self.lengths[sid]:
+            raise InvalidArgument("only full blocks can be registered")
+        new = 0
+        for b, k in zip(self.tables[sid], keys):
+            if k in self.block_of or b in self.key_of:
+                continue
+            self.block_of[k] = b
+            self.key_of[b] = k
+            new += 1
+        return new
+
+    def seq_add_cached(self, keys):
+        """New sequence sharing the registered blocks of its leading keys; (sid, hits)."""
+        sid = self.seq_add()
+        table = self.tables[sid]
+        for k in keys:
+            b = self.block_of.get(int(k))
+            if b is None:
+                break
+            if self.refcount[b] == 0:
+                del self.evictable[b]
+            self.refcount[b] += 1
+            table.append(b)
+        self.lengths[sid] = len(table) * self.block_size
+        return sid, len(table)
 
     # ---- views ---------------------------------------------------------------
     def table(self, sid: int) -> list[int]:

@@ -122,10 +122,10 @@ def pa_num_free_blocks(pool) -> int:
 
 def pa_free_list(pool) -> np.ndarray:
     """Free stack bottom first: the last entry is handed out next."""
-    n = pa_num_free_blocks(pool)
-    out = np.empty(n, np.int32)
     got = ctypes.c_int32()
-    _check(_lib().pa_free_list(pool, out.ctypes.data, n, ctypes.byref(got)))
+    _check(_lib().pa_free_list(pool, None, 0, ctypes.byref(got)))
+    out = np.empty(got.value, np.int32)
+    _check(_lib().pa_free_list(pool, out.ctypes.data, got.value, ctypes.byref(got)))
     return out
 
 
@@ -187,6 +187,32 @@ def pa_build_block_tables(pool, seq_ids, max_blocks: int, tables_out=None, lens_
     _check(_lib().pa_build_block_tables(pool, ids.ctypes.data, n, max_blocks, _host_ptr(tables),
                                         _host_ptr(lens)))
     return tables, lens
+
+
+# ------------------------------------------------------------------ prefix caching
+def pa_prefix_register(pool, seq_id: int, keys) -> int:
+    """Register the first len(keys) (full) blocks of seq_id under keys; returns how many were new."""
+    k = np.ascontiguousarray(keys, dtype=np.uint64)
+    n = ctypes.c_int32()
+    _check(_lib().pa_prefix_register(pool, seq_id, k.ctypes.data, k.shape[0], ctypes.byref(n)))
+    return n.value
+
+
+def pa_seq_add_cached(pool, keys):
+    """New sequence sharing the registered blocks of its leading keys: (seq_id, hits)."""
+    k = np.ascontiguousarray(keys, dtype=np.uint64)
+    sid, hit = ctypes.c_int32(), ctypes.c_int32()
+    _check(_lib().pa_seq_add_cached(pool, k.ctypes.data, k.shape[0], ctypes.byref(sid), ctypes.byref(hit)))
+    return sid.value, hit.value
+
+
+def pa_prefix_evictable(pool) -> np.ndarray:
+    """Evictable cached blocks, next to be evicted first."""
+    n = ctypes.c_int32()
+    _check(_lib().pa_prefix_evictable(pool, None, 0, ctypes.byref(n)))
+    out = np.empty(n.value, np.int32)
+    _check(_lib().pa_prefix_evictable(pool, out.ctypes.data, n.value, ctypes.byref(n)))
+    return out
 
 
 # ------------------------------------------------------------------ device work

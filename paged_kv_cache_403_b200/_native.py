@@ -21,7 +21,8 @@ class PoolConfig(ctypes.Structure):
 class PoolStats(ctypes.Structure):
     _fields_ = [("num_blocks", c_i32), ("num_free", c_i32), ("num_shared", c_i32),
                 ("num_seqs", c_i32), ("num_tokens", c_i64), ("cow_copies", c_i64),
-                ("peak_used", c_i32)]
+                ("peak_used", c_i32), ("num_cached", c_i32), ("num_evictable", c_i32),
+                ("cache_hits", c_i64), ("cache_evictions", c_i64)]
 
 
 # name -> (restype, argtypes); every function declared in include/pa.h
@@ -44,6 +45,9 @@ SIGNATURES = {
     "pa_seq_info": (ctypes.c_int, [c_vp, c_i32, P_i32, c_vp, c_i32, P_i32]),
     "pa_reserve_slots": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, P_i32]),
     "pa_build_block_tables": (ctypes.c_int, [c_vp, c_vp, c_i32, c_i32, c_vp, c_vp]),
+    "pa_prefix_register": (ctypes.c_int, [c_vp, c_i32, c_vp, c_i32, P_i32]),
+    "pa_seq_add_cached": (ctypes.c_int, [c_vp, c_vp, c_i32, P_i32, P_i32]),
+    "pa_prefix_evictable": (ctypes.c_int, [c_vp, c_vp, c_i32, P_i32]),
     "pa_copy_blocks": (ctypes.c_int, [c_vp, c_vp, c_i32, c_vp]),
     "pa_append_kv": (ctypes.c_int, [c_vp, c_i32, c_vp, c_vp, c_vp, c_i32, c_vp]),
     "pa_decode_max_splits": (c_i32, [c_i32, c_i32, c_i32]),

@@ -45,20 +45,75 @@ bool drop_ref(pa_pool *p, int32_t b) {
 }
 
 void note_usage(pa_pool *p) {
-    int32_t used = p->cfg.num_blocks - (int32_t)p->free_stack.size();
+    int32_t used = p->cfg.num_blocks - (int32_t)p->free_stack.size() - p->ev_count;
     p->peak_used = std::max(p->peak_used, used);
 }
 
-pa_status pop_block(pa_pool *p, int32_t *b) {
+// ---- evictable queue (registered blocks with refcount 0), oldest at the head
+void ev_push_back(pa_pool *p, int32_t b) {
+    p->ev_prev[b] = p->ev_tail;
+    p->ev_next[b] = -1;
+    if (p->ev_tail >= 0) p->ev_next[p->ev_tail] = b; else p->ev_head = b;
+    p->ev_tail = b;
+    p->in_ev[b] = 1;
+    ++p->ev_count;
+}
+
+void ev_push_front(pa_pool *p, int32_t b) {
+    p->ev_prev[b] = -1;
+    p->ev_next[b] = p->ev_head;
+    if (p->ev_head >= 0) p->ev_prev[p->ev_head] = b; else p->ev_tail = b;
+    p->ev_head = b;
+    p->in_ev[b] = 1;
+    ++p->ev_count;
+}
+
+void ev_unlink(pa_pool *p, int32_t b) {
+    const int32_t pr = p->ev_prev[b], nx = p->ev_next[b];
+    if (pr >= 0) p->ev_next[pr] = nx; else p->ev_head = nx;
+    if (nx >= 0) p->ev_prev[nx] = pr; else p->ev_tail = pr;
+    p->in_ev[b] = 0;
+    --p->ev_count;
+}
+
+void unregister(pa_pool *p, int32_t b) {
+    p->block_of.erase(p->key_of[b]);
+    p->has_key[b] = 0;
+}
+
+void register_key(pa_pool *p, int32_t b, uint64_t key) {
+    p->block_of.emplace(key, b);
+    p->key_of[b] = key;
+    p->has_key[b] = 1;
+}
+
+// A block whose last reference went away: cached blocks stay findable in the queue.
+void release(pa_pool *p, int32_t b) {
+    if (p->has_key[b]) ev_push_back(p, b); else p->free_stack.push_back(b);
+}
+
+// Take a block: the free stack first, else evict the least recently released cached
+// block.  *evicted_key is set (and *was_evicted true) when a cached block was reclaimed.
+pa_status pop_block(pa_pool *p, int32_t *b, bool *was_evicted, uint64_t *evicted_key) {
+    *was_evicted = false;
     if (p->fail_alloc_after == 0) {
         p->fail_alloc_after = -1;
         return fail(PA_ERR_OUT_OF_BLOCKS, "block allocation failed (injected)");
     }
-    if (p->free_stack.empty())
+    if (p->free_stack.empty() && p->ev_head < 0)
         return fail(PA_ERR_OUT_OF_BLOCKS, "no free KV blocks left in the pool");
     if (p->fail_alloc_after > 0) --p->fail_alloc_after;
-    *b = p->free_stack.back();
-    p->free_stack.pop_back();
+    if (!p->free_stack.empty()) {
+        *b = p->free_stack.back();
+        p->free_stack.pop_back();
+    } else {
+        *b = p->ev_head;
+        ev_unlink(p, *b);
+        *was_evicted = true;
+        *evicted_key = p->key_of[*b];
+        unregister(p, *b);
+        ++p->cache_evictions;
+    }
     p->refcount[*b] = 1;
     return PA_OK;
 }
@@ -66,10 +121,11 @@ pa_status pop_block(pa_pool *p, int32_t *b) {
 // Undo journal for pa_reserve_slots: every mutation is recorded and replayed
 // backwards if the call runs out of blocks part way.
 struct Undo {
-    enum Kind { kAlloc, kDrop, kPush, kSet, kLen, kCow } kind;
+    enum Kind { kAlloc, kEvict, kDrop, kPush, kSet, kLen, kCow } kind;
     int32_t seq;
     int32_t a;
     int32_t b;
+    uint64_t key;
 };
 
 }  // namespace
@@ -110,6 +166,11 @@ pa_status pa_pool_create(const pa_pool_config *cfg, void *k_pool, void *v_pool,
     p->v_pool = v_pool;
     const int32_t nb = cfg->num_blocks;
     p->refcount.assign(nb, 0);
+    p->key_of.assign(nb, 0);
+    p->has_key.assign(nb, 0);
+    p->ev_prev.assign(nb, -1);
+    p->ev_next.assign(nb, -1);
+    p->in_ev.assign(nb, 0);
     p->free_stack.resize(nb);
     if (free_order) {
         std::vector<char> seen(nb, 0);
@@ -138,18 +199,24 @@ pa_status pa_pool_destroy(pa_pool *pool) {
 pa_status pa_pool_stats(const pa_pool *p, pa_pool_stats_t *o) {
     if (!p || !o) return fail(PA_ERR_INVALID_ARG, "pa_pool_stats: null argument");
     o->num_blocks = p->cfg.num_blocks;
-    o->num_free = (int32_t)p->free_stack.size();
+    o->num_free = (int32_t)p->free_stack.size() + p->ev_count;
     o->num_shared = p->num_shared;
     o->num_seqs = (int32_t)p->seqs.size();
     o->num_tokens = p->num_tokens;
     o->cow_copies = p->cow_copies;
     o->peak_used = p->peak_used;
+    o->num_cached = (int32_t)p->block_of.size();
+    o->num_evictable = p->ev_count;
+    o->cache_hits = p->cache_hits;
+    o->cache_evictions = p->cache_evictions;
     return PA_OK;
 }
 
 pa_status pa_alloc_block(pa_pool *p, int32_t *block) {
     if (!p || !block) return fail(PA_ERR_INVALID_ARG, "pa_alloc_block: null argument");
-    pa_status st = pop_block(p, block);
+    bool ev;
+    uint64_t key;
+    pa_status st = pop_block(p, block, &ev, &key);
     if (st == PA_OK) note_usage(p);
     return st;
 }
@@ -158,7 +225,7 @@ pa_status pa_free_block(pa_pool *p, int32_t block) {
     if (!p || !valid_block(p, block)) return fail(PA_ERR_INVALID_ARG, "pa_free_block: bad block id");
     if (p->refcount[block] == 0)
         return fail(PA_ERR_DOUBLE_FREE, "pa_free_block: block " + std::to_string(block) + " is already free");
-    if (drop_ref(p, block)) p->free_stack.push_back(block);
+    if (drop_ref(p, block)) release(p, block);
     return PA_OK;
 }
 
@@ -177,7 +244,7 @@ pa_status pa_block_refcount(const pa_pool *p, int32_t block, int32_t *rc) {
 
 pa_status pa_num_free_blocks(const pa_pool *p, int32_t *n) {
     if (!p || !n) return fail(PA_ERR_INVALID_ARG, "pa_num_free_blocks: null argument");
-    *n = (int32_t)p->free_stack.size();
+    *n = (int32_t)p->free_stack.size() + p->ev_count;
     return PA_OK;
 }
 
@@ -221,7 +288,7 @@ pa_status pa_seq_free(pa_pool *p, int32_t seq_id) {
     auto it = p->seqs.find(seq_id);
     if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_seq_free: unknown sequence");
     for (int32_t b : it->second.table)
-        if (drop_ref(p, b)) p->free_stack.push_back(b);
+        if (drop_ref(p, b)) release(p, b);
     p->num_tokens -= it->second.len;
     p->seqs.erase(it);
     return PA_OK;
@@ -274,36 +341,38 @@ pa_status pa_reserve_slots(pa_pool *p, const int32_t *seq_ids, const int32_t *nt
         pa_pool::Seq &s = *seqs[i];
         for (int32_t t = 0; t < ntok[i]; ++t) {
             const int32_t L = s.len;
+            bool ev;
+            uint64_t key;
             if (L % B == 0) {
                 int32_t b;
-                st = pop_block(p, &b);
+                st = pop_block(p, &b, &ev, &key);
                 if (st != PA_OK) break;
-                journal.push_back({Undo::kAlloc, seq_ids[i], b, 0});
+                journal.push_back({ev ? Undo::kEvict : Undo::kAlloc, seq_ids[i], b, 0, key});
                 s.table.push_back(b);
-                journal.push_back({Undo::kPush, seq_ids[i], 0, 0});
+                journal.push_back({Undo::kPush, seq_ids[i], 0, 0, 0});
             } else {
                 const int32_t tail = s.table.back();
                 if (p->refcount[tail] > 1) {
                     int32_t nb;
-                    st = pop_block(p, &nb);
+                    st = pop_block(p, &nb, &ev, &key);
                     if (st != PA_OK) break;
-                    journal.push_back({Undo::kAlloc, seq_ids[i], nb, 0});
+                    journal.push_back({ev ? Undo::kEvict : Undo::kAlloc, seq_ids[i], nb, 0, key});
                     drop_ref(p, tail);
-                    journal.push_back({Undo::kDrop, seq_ids[i], tail, 0});
+                    journal.push_back({Undo::kDrop, seq_ids[i], tail, 0, 0});
                     const int32_t idx = (int32_t)s.table.size() - 1;
                     s.table[idx] = nb;
-                    journal.push_back({Undo::kSet, seq_ids[i], idx, tail});
+                    journal.push_back({Undo::kSet, seq_ids[i], idx, tail, 0});
                     if (cow_pairs_out) {
                         cow_pairs_out[2 * cows] = tail;
                         cow_pairs_out[2 * cows + 1] = nb;
                     }
                     ++cows;
-                    journal.push_back({Undo::kCow, seq_ids[i], 0, 0});
+                    journal.push_back({Undo::kCow, seq_ids[i], 0, 0, 0});
                 }
             }
             slot_mapping_out[k++] = (int64_t)s.table[L / B] * B + L % B;
             s.len = L + 1;
-            journal.push_back({Undo::kLen, seq_ids[i], L, 0});
+            journal.push_back({Undo::kLen, seq_ids[i], L, 0, 0});
         }
     }
     if (st != PA_OK) {
@@ -314,6 +383,12 @@ pa_status pa_reserve_slots(pa_pool *p, const int32_t *seq_ids, const int32_t *nt
             case Undo::kAlloc:
                 p->refcount[it->a] = 0;
                 p->free_stack.push_back(it->a);
+                break;
+            case Undo::kEvict:   // it was the head of the queue when it was taken
+                p->refcount[it->a] = 0;
+                register_key(p, it->a, it->key);
+                ev_push_front(p, it->a);
+                --p->cache_evictions;
                 break;
             case Undo::kDrop: add_ref(p, it->a); break;
             case Undo::kPush: s.table.pop_back(); break;
@@ -349,6 +424,56 @@ pa_status pa_build_block_tables(const pa_pool *p, const int32_t *seq_ids, int32_
         std::fill(row + nb, row + max_blocks, -1);
         lens_out[i] = s.len;
     }
+    return PA_OK;
+}
+
+pa_status pa_prefix_register(pa_pool *p, int32_t seq_id, const uint64_t *keys, int32_t n_blocks,
+                             int32_t *n_new) {
+    if (!p || n_blocks < 0 || (n_blocks > 0 && !keys)) return fail(PA_ERR_INVALID_ARG, "pa_prefix_register: bad argument");
+    auto it = p->seqs.find(seq_id);
+    if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_prefix_register: unknown sequence");
+    const pa_pool::Seq &s = it->second;
+    if ((int64_t)n_blocks * p->cfg.block_size > s.len)
+        return fail(PA_ERR_INVALID_ARG, "pa_prefix_register: only full blocks can be registered");
+    int32_t added = 0;
+    for (int32_t i = 0; i < n_blocks; ++i) {
+        const int32_t b = s.table[i];
+        if (p->has_key[b] || p->block_of.count(keys[i])) continue;
+        register_key(p, b, keys[i]);
+        ++added;
+    }
+    if (n_new) *n_new = added;
+    return PA_OK;
+}
+
+pa_status pa_seq_add_cached(pa_pool *p, const uint64_t *keys, int32_t n_keys, int32_t *seq_id, int32_t *n_hit) {
+    if (!p || !seq_id || !n_hit || n_keys < 0 || (n_keys > 0 && !keys))
+        return fail(PA_ERR_INVALID_ARG, "pa_seq_add_cached: bad argument");
+    if (p->next_seq == INT32_MAX) return fail(PA_ERR_INVALID_ARG, "pa_seq_add_cached: sequence ids exhausted");
+    pa_pool::Seq s;
+    for (int32_t i = 0; i < n_keys; ++i) {
+        auto f = p->block_of.find(keys[i]);
+        if (f == p->block_of.end()) break;
+        const int32_t b = f->second;
+        if (p->refcount[b] == 0) ev_unlink(p, b);
+        add_ref(p, b);
+        s.table.push_back(b);
+    }
+    s.len = (int32_t)s.table.size() * p->cfg.block_size;
+    *n_hit = (int32_t)s.table.size();
+    *seq_id = p->next_seq++;
+    p->num_tokens += s.len;
+    p->cache_hits += *n_hit;
+    p->seqs.emplace(*seq_id, std::move(s));
+    note_usage(p);
+    return PA_OK;
+}
+
+pa_status pa_prefix_evictable(const pa_pool *p, int32_t *out, int32_t cap, int32_t *n) {
+    if (!p || !n || (cap > 0 && !out)) return fail(PA_ERR_INVALID_ARG, "pa_prefix_evictable: bad argument");
+    *n = p->ev_count;
+    int32_t k = 0;
+    for (int32_t b = p->ev_head; b >= 0 && k < cap; b = p->ev_next[b]) out[k++] = b;
     return PA_OK;
 }
 

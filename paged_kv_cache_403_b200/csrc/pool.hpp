@@ -33,6 +33,17 @@ struct pa_pool {
     int32_t peak_used = 0;
     int64_t fail_alloc_after = -1;    // host fault injection (< 0: off)
 
+    // Prefix caching: registered full blocks (key <-> block) and the queue of
+    // registered blocks whose refcount fell to zero, least recently released first
+    // (an intrusive doubly linked list over block ids).
+    std::unordered_map<uint64_t, int32_t> block_of;
+    std::vector<uint64_t> key_of;
+    std::vector<char> has_key;
+    std::vector<int32_t> ev_prev, ev_next;
+    std::vector<char> in_ev;
+    int32_t ev_head = -1, ev_tail = -1, ev_count = 0;
+    int64_t cache_hits = 0, cache_evictions = 0;
+
     // TMA descriptors over the whole key / value pools, viewed as 2-D tensors of
     // [num_layers * num_blocks * num_kv_heads * block_size rows][head_dim]; built on
     // the first decode call (16-bit caches only).

@@ -193,3 +193,75 @@ class ContinuousBatch:
         self.retire(self.t)
         self.t += 1
         return rec
+
+
+class SharedPromptBatch(ContinuousBatch):
+    """Continuous batch whose prompts share a system prompt; with ``cache`` the system
+    prompt's full blocks are registered once and every later admission shares them
+    (pa_seq_add_cached) and appends only its own suffix."""
+
+    def __init__(self, recipe, device="cuda", max_blocks=None, cache=True):
+        from synthetic.workloads import prompt_rows, system_block_keys
+        self._rows, self.cache_on = prompt_rows, cache
+        self.recipe = recipe
+        self.shape = shape = recipe["shape"]
+        self.sched = recipe["schedule"]
+        self.system, self.system_uid = recipe["system"], recipe["system_uid"]
+        self.keys = system_block_keys(self.system // shape.block_size, self.system_uid)
+        self.cache = PagedCache.from_shape(shape, recipe["order"], device)
+        self.gen = DeviceGen(recipe["seed"], shape, device)
+        self.device = device
+        n = len(self.sched.initial)
+        self.sids, self.uids = [None] * n, list(range(n))
+        self.appended_rows = 0
+        init = [int(L) for L in self.sched.initial]
+        # the first request writes (and registers) the system prompt; the rest can share it
+        self._admit_many([0], [0], init[:1])
+        if n > 1:
+            self._admit_many(list(range(1, n)), list(range(1, n)), init[1:])
+        self.next_uid = n
+        self.max_blocks = max_blocks or -(-(4096 + len(self.sched.events) + 1) // shape.block_size)
+        self.pending = []
+        self.t = 0
+
+    def _admit_many(self, slots, uids, lens):
+        from paged_kv_cache_403_b200 import pa_prefix_register, pa_seq_add_cached
+        pool = self.cache.pool
+        starts = []
+        for slot, uid, plen in zip(slots, uids, lens):
+            if self.cache_on:
+                sid, hit = pa_seq_add_cached(pool, self.keys)
+            else:
+                sid, hit = self.cache.add(), 0
+            self.sids[slot] = sid
+            starts.append(hit * self.shape.block_size)
+        sids = [self.sids[s] for s in slots]
+        ntok = [plen - st for plen, st in zip(lens, starts)]
+        slots_host, cow = self.cache.reserve(sids, ntok)
+        assert len(cow) == 0
+        ru, rt = zip(*[self._rows(u, p, self.system, self.system_uid, st) for u, p, st in zip(uids, lens, starts)])
+        ru, rt = np.concatenate(ru), np.concatenate(rt)
+        dev = torch.from_numpy(np.ascontiguousarray(slots_host)).to(self.device)
+        for lo in range(0, len(ru), 1 << 16):
+            hi = min(len(ru), lo + (1 << 16))
+            for layer in range(self.cache.num_layers):
+                k, v = self.gen.kv(layer, ru[lo:hi], rt[lo:hi])
+                self.cache.append(layer, k, v, dev[lo:hi])
+        self.appended_rows += len(ru)
+        if self.cache_on:
+            for sid, st in zip(sids, starts):
+                if st == 0:                      # first writer of the system prompt registers it
+                    pa_prefix_register(pool, sid, self.keys)
+
+    def admit(self):
+        if not self.pending:
+            return []
+        slots = [s for s, _ in self.pending]
+        uids = list(range(self.next_uid, self.next_uid + len(slots)))
+        lens = [p for _, p in self.pending]
+        for s, u in zip(slots, uids):
+            self.uids[s] = u
+        self.next_uid += len(slots)
+        self._admit_many(slots, uids, lens)
+        self.pending = []
+        return list(zip([self.sids[s] for s in slots], uids, lens))

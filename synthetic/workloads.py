@@ -115,3 +115,32 @@ def large_pool(seed: int = 5, block_size: int = 16, n: int = 384, num_layers: in
     shape = Shape(num_layers, block_size, 32, 8, 128, "f16", nb, kv_scale=1.0 / math.sqrt(128.0))
     order = np.random.default_rng(seed + 1000 * block_size).permutation(nb).astype(np.int32)
     return dict(name=f"large_pool_b{block_size}", seed=seed, shape=shape, lens=lens, order=order)
+
+
+SYSTEM_UID = (1 << 22) - 1   # writer uid of the shared system prompt's keys and values
+
+
+def shared_prompt_batch(seed: int = 6, n: int = 256, steps: int = 64, system: int = 1024,
+                        p_stop: float = 1.0 / 200.0) -> dict:
+    """Continuous batch whose prompts all start with the same `system`-token prompt:
+    prompt lengths U[system + 128, 4096]; positions < system are written by
+    SYSTEM_UID (identical in every request), later ones by the request's own uid.
+    Block 16, 32 q / 8 KV heads, d128, bf16."""
+    shape = Shape(1, 16, 32, 8, 128, "bf16",
+                  num_blocks=n * ((4096 + max(steps, 64) + 15) // 16), kv_scale=1.0 / math.sqrt(128.0))
+    order = np.random.default_rng(seed + 1000).permutation(shape.num_blocks).astype(np.int32)
+    return dict(name="shared_prompt", seed=seed, shape=shape, order=order, system=system,
+                system_uid=SYSTEM_UID,
+                schedule=continuous_schedule(n, steps, seed, system + 128, 4096, p_stop))
+
+
+def prompt_rows(uid: int, plen: int, system: int = 0, system_uid: int = SYSTEM_UID, start: int = 0):
+    """(writer uid, token) of prompt positions start..plen-1: the shared system prompt
+    for positions < system, the request itself after."""
+    pos = np.arange(start, plen)
+    return np.where(pos < system, system_uid, uid), pos
+
+
+def system_block_keys(n_blocks: int, system_uid: int = SYSTEM_UID):
+    """Cache keys of the shared system prompt's full blocks (stand-in for a hash chain)."""
+    return [(system_uid << 32) | i for i in range(n_blocks)]

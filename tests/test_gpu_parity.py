@@ -227,3 +227,35 @@ def test_large_pool_sampled(bs, split):
             check_close(out[i], ref, "f16", "f16", f"layer {layer} seq {i}")
     del cache
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ prefix caching on the GPU
+@pytest.mark.parametrize("cache_on", [True, False])
+def test_shared_prompt_with_prefix_cache(cache_on):
+    """Requests share a 256-token system prompt; with the cache its 16 blocks are written
+    once and shared by every later admission.  Attention over the shared blocks matches
+    the oracle on each request's regenerated history (system prompt + own tokens)."""
+    from paged_kv_cache_403_b200.runners import SharedPromptBatch
+    r = wl.shared_prompt_batch(seed=61, n=12, steps=6, system=256, p_stop=0.15)
+    sh, sysl, sys_uid = r["shape"], r["system"], r["system_uid"]
+    sb = SharedPromptBatch(r, max_blocks=272, cache=cache_on)
+    st = pa.pa_pool_stats(sb.cache.pool)
+    if cache_on:
+        assert st["num_cached"] == sysl // 16 and st["cache_hits"] == (12 - 1) * (sysl // 16)
+    else:
+        assert st["num_cached"] == 0
+    for t in range(6):
+        rec = sb.step(split_tokens=512, out_dtype=torch.float32)
+        out = widen(rec.outputs[0])
+        for i in range(len(rec.lens)):
+            uid = rec.uids[i]
+            ref = sequence_attention(sh, r["seed"], 0, uid, int(rec.lens[i]), uid, int(rec.positions[i]),
+                                     writer=lambda p, u=uid: (sys_uid, p) if p < sysl else (u, p))
+            check_close(out[i], ref, "f32", "bf16", f"step {t} seq {i}")
+        if cache_on:   # every live sequence starts with the same 16 physical blocks
+            first = {tuple(row[:sysl // 16]) for row in rec.tables}
+            assert len(first) == 1
+    admitted = sum(len(e) for e in r["schedule"].events[:5])
+    assert admitted > 0
+    if cache_on:
+        assert pa.pa_pool_stats(sb.cache.pool)["cache_hits"] == (12 - 1 + admitted) * (sysl // 16)
