@@ -189,6 +189,27 @@ pa_status pa_seq_add_cached(pa_pool *pool, const uint64_t *keys, int32_t n_keys,
  * *n receives its length. */
 pa_status pa_prefix_evictable(const pa_pool *pool, int32_t *out, int32_t cap, int32_t *n);
 
+/* ------------------------------------------------------------------ preemption with swap */
+
+/* [P1] "The senior-level nuance" / "What happens when the KV cache is full?": a full
+ * pool must queue, preempt, offload cache data or reject.  These calls offload one
+ * sequence's cache to host memory and bring it back.
+ * Host buffer layout (caller-owned, page-locked so the GPU can reach it, e.g. from
+ * cudaHostAlloc): [block i in logical order][layer][K, V][num_kv_heads][block_size]
+ * [head_dim] of the pool dtype; pa_swap_bytes gives its size. */
+pa_status pa_swap_bytes(const pa_pool *pool, int32_t seq_id, size_t *bytes);
+/* Enqueue on `stream` a copy of every block of seq_id (all layers, K and V) into
+ * host_buf, then drop one reference on each block (logical order), as a retire does.
+ * The sequence keeps its id and length but owns no blocks until pa_swap_in; appends,
+ * forks and tables are refused for it meanwhile.  Later device work that reuses the
+ * freed blocks must be issued on the same stream (or ordered after it).  A pool
+ * without device memory does the bookkeeping only (host_buf may be NULL). */
+pa_status pa_swap_out(pa_pool *pool, int32_t seq_id, void *host_buf, size_t buf_bytes, pa_stream stream);
+/* Take ceil(length / block_size) blocks (one allocation after the other, as appends
+ * would), make them the sequence's table and enqueue on `stream` the copy of host_buf
+ * back into them.  PA_ERR_OUT_OF_BLOCKS leaves everything unchanged. */
+pa_status pa_swap_in(pa_pool *pool, int32_t seq_id, const void *host_buf, size_t buf_bytes, pa_stream stream);
+
 /* ------------------------------------------------------------------ device work */
 
 /* Copy-on-write block copies: for each pair (src, dst) in pairs_dev[n_pairs][2]

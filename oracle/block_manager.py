@@ -54,6 +54,16 @@ pages give no lookup, so the reading taken is:
 10. a new sequence built from keys walks them in order and shares each
    registered block (count + 1, leaving the queue if it was there) until the
    first miss; its length is then (hits x B).
+
+Preemption with swap (page 1, "The senior-level nuance" and "What happens when
+the KV cache is full?": a full pool must queue, preempt, offload or reject):
+
+11. swapping a sequence out copies its blocks, in logical order, to host memory
+   and then drops one reference on each of them (logical order, as a retire
+   does); the sequence keeps its id and length but owns no block.
+12. swapping it back in takes ceil(L / B) blocks from the allocator one after
+   the other (as appends would) and copies the data back in logical order; if
+   the pool cannot supply them all, nothing changes.
 """
 from __future__ import annotations
 
@@ -90,6 +100,7 @@ class BlockManagerModel:
         self.key_of: dict[int, int] = {}            # block -> key (registered blocks)
         self.block_of: dict[int, int] = {}          # key -> block
         self.evictable: OrderedDict = OrderedDict()  # registered blocks with count 0, oldest first
+        self.swapped: set[int] = set()              # sequences whose blocks are in host memory
 
     # ---- blocks --------------------------------------------------------------
     def num_free(self) -> int:
@@ -136,7 +147,7 @@ class BlockManagerModel:
         return sid
 
     def seq_fork(self, parent: int) -> int:
-        if parent not in self.tables:
+        if parent not in self.tables or parent in self.swapped:
             raise InvalidArgument(parent)
         child = self.seq_add()
         for b in self.tables[parent]:
@@ -152,6 +163,7 @@ class BlockManagerModel:
             self.free(b)
         del self.tables[sid]
         del self.lengths[sid]
+        self.swapped.discard(sid)
 
     def _append_one(self, sid: int, cow_pairs: list) -> int:
         B = self.block_size
@@ -180,7 +192,7 @@ class BlockManagerModel:
         if len(seq_ids) != len(ntok) or len(set(seq_ids)) != len(seq_ids):
             raise InvalidArgument("seq_ids must be distinct and match ntok")
         for s, n in zip(seq_ids, ntok):
-            if s not in self.tables or n < 0:
+            if s not in self.tables or n < 0 or s in self.swapped:
                 raise InvalidArgument(s)
         saved = copy.deepcopy((self.free_stack, self.refcount, self.tables, self.lengths, self.key_of,
                                self.block_of, self.evictable))
@@ -227,6 +239,33 @@ class BlockManagerModel:
             table.append(b)
         self.lengths[sid] = len(table) * self.block_size
         return sid, len(table)
+
+    # ---- preemption with swap ---------------------------------------------------
+    def swap_out(self, sid: int):
+        """Returns the blocks whose contents go to host memory (logical order)."""
+        if sid not in self.tables or sid in self.swapped:
+            raise InvalidArgument(sid)
+        blocks = list(self.tables[sid])
+        for b in blocks:
+            self.free(b)
+        self.tables[sid] = []
+        self.swapped.add(sid)
+        return blocks
+
+    def swap_in(self, sid: int):
+        """Returns the new blocks the host copy is written back to (logical order)."""
+        if sid not in self.swapped:
+            raise InvalidArgument(sid)
+        n = -(-self.lengths[sid] // self.block_size)
+        saved = copy.deepcopy((self.free_stack, self.refcount, self.key_of, self.block_of, self.evictable))
+        try:
+            blocks = [self.alloc() for _ in range(n)]
+        except OutOfBlocks:
+            self.free_stack, self.refcount, self.key_of, self.block_of, self.evictable = saved
+            raise
+        self.tables[sid] = blocks
+        self.swapped.discard(sid)
+        return blocks
 
     # ---- views ---------------------------------------------------------------
     def table(self, sid: int) -> list[int]:

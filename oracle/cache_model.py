@@ -47,3 +47,19 @@ def copy_blocks(k_pool, v_pool, pairs):
     for src, dst in pairs:
         k_pool[:, int(dst)] = k_pool[:, int(src)]
         v_pool[:, int(dst)] = v_pool[:, int(src)]
+
+
+def swap_buffer(k_pool, v_pool, blocks):
+    """Host copy of a swapped-out sequence: [block i][layer][K, V][heads][block_size][dim]
+    (reading: block-major so one block's data is contiguous and can be restored into
+    any free block)."""
+    parts = [np.stack([k_pool[:, int(b)], v_pool[:, int(b)]], axis=1) for b in blocks]
+    return np.ascontiguousarray(np.stack(parts)) if parts else np.zeros((0,) + k_pool.shape[:1] + (2,)
+                                                                          + k_pool.shape[2:], k_pool.dtype)
+
+
+def swap_restore(k_pool, v_pool, blocks, buf):
+    """Write a swap buffer back into the given (new) blocks, logical order."""
+    for i, b in enumerate(blocks):
+        k_pool[:, int(b)] = buf[i, :, 0]
+        v_pool[:, int(b)] = buf[i, :, 1]

@@ -215,6 +215,32 @@ def pa_prefix_evictable(pool) -> np.ndarray:
     return out
 
 
+# ------------------------------------------------------------------ preemption with swap
+def pa_swap_bytes(pool, seq_id: int) -> int:
+    n = ctypes.c_size_t()
+    _check(_lib().pa_swap_bytes(pool, seq_id, ctypes.byref(n)))
+    return n.value
+
+
+def _swap_buf(host_buf):
+    if host_buf is None:
+        return None, 0
+    assert not host_buf.is_cuda and host_buf.is_pinned() and host_buf.is_contiguous()
+    return host_buf.data_ptr(), host_buf.numel() * host_buf.element_size()
+
+
+def pa_swap_out(pool, seq_id: int, host_buf=None, stream=None) -> None:
+    """Copy seq_id's blocks to the pinned CPU tensor host_buf and release them."""
+    ptr, nbytes = _swap_buf(host_buf)
+    _check(_lib().pa_swap_out(pool, seq_id, ptr, nbytes, _stream(stream) if ptr else None))
+
+
+def pa_swap_in(pool, seq_id: int, host_buf=None, stream=None) -> None:
+    """Give seq_id new blocks and copy host_buf back into them."""
+    ptr, nbytes = _swap_buf(host_buf)
+    _check(_lib().pa_swap_in(pool, seq_id, ptr, nbytes, _stream(stream) if ptr else None))
+
+
 # ------------------------------------------------------------------ device work
 def pa_copy_blocks(pool, pairs_dev, n_pairs=None, stream=None) -> None:
     n = pairs_dev.shape[0] if n_pairs is None else n_pairs

@@ -48,6 +48,9 @@ SIGNATURES = {
     "pa_prefix_register": (ctypes.c_int, [c_vp, c_i32, c_vp, c_i32, P_i32]),
     "pa_seq_add_cached": (ctypes.c_int, [c_vp, c_vp, c_i32, P_i32, P_i32]),
     "pa_prefix_evictable": (ctypes.c_int, [c_vp, c_vp, c_i32, P_i32]),
+    "pa_swap_bytes": (ctypes.c_int, [c_vp, c_i32, ctypes.POINTER(c_sz)]),
+    "pa_swap_out": (ctypes.c_int, [c_vp, c_i32, c_vp, c_sz, c_vp]),
+    "pa_swap_in": (ctypes.c_int, [c_vp, c_i32, c_vp, c_sz, c_vp]),
     "pa_copy_blocks": (ctypes.c_int, [c_vp, c_vp, c_i32, c_vp]),
     "pa_append_kv": (ctypes.c_int, [c_vp, c_i32, c_vp, c_vp, c_vp, c_i32, c_vp]),
     "pa_decode_max_splits": (c_i32, [c_i32, c_i32, c_i32]),

@@ -274,6 +274,7 @@ pa_status pa_seq_fork(pa_pool *p, int32_t parent, int32_t *child) {
     if (!p || !child) return fail(PA_ERR_INVALID_ARG, "pa_seq_fork: null argument");
     auto it = p->seqs.find(parent);
     if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_seq_fork: unknown parent");
+    if (it->second.swapped) return fail(PA_ERR_INVALID_ARG, "pa_seq_fork: parent is swapped out");
     if (p->next_seq == INT32_MAX) return fail(PA_ERR_INVALID_ARG, "pa_seq_fork: sequence ids exhausted");
     pa_pool::Seq s = it->second;          // copy of table and length
     for (int32_t b : s.table) add_ref(p, b);
@@ -319,6 +320,7 @@ pa_status pa_reserve_slots(pa_pool *p, const int32_t *seq_ids, const int32_t *nt
         auto it = p->seqs.find(seq_ids[i]);
         if (it == p->seqs.end() || ntok[i] < 0)
             return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: unknown sequence or negative count");
+        if (it->second.swapped) return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: sequence is swapped out");
         if ((int64_t)it->second.len + ntok[i] > INT32_MAX)
             return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: sequence too long");
         seqs[i] = &it->second;
@@ -413,6 +415,7 @@ pa_status pa_build_block_tables(const pa_pool *p, const int32_t *seq_ids, int32_
     for (int32_t i = 0; i < n; ++i) {
         auto it = p->seqs.find(seq_ids[i]);
         if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_build_block_tables: unknown sequence");
+        if (it->second.swapped) return fail(PA_ERR_INVALID_ARG, "pa_build_block_tables: sequence is swapped out");
         if ((int32_t)it->second.table.size() > max_blocks)
             return fail(PA_ERR_INVALID_ARG, "pa_build_block_tables: sequence has more than max_blocks blocks");
     }
@@ -432,6 +435,7 @@ pa_status pa_prefix_register(pa_pool *p, int32_t seq_id, const uint64_t *keys, i
     if (!p || n_blocks < 0 || (n_blocks > 0 && !keys)) return fail(PA_ERR_INVALID_ARG, "pa_prefix_register: bad argument");
     auto it = p->seqs.find(seq_id);
     if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_prefix_register: unknown sequence");
+    if (it->second.swapped) return fail(PA_ERR_INVALID_ARG, "pa_prefix_register: sequence is swapped out");
     const pa_pool::Seq &s = it->second;
     if ((int64_t)n_blocks * p->cfg.block_size > s.len)
         return fail(PA_ERR_INVALID_ARG, "pa_prefix_register: only full blocks can be registered");
@@ -474,6 +478,88 @@ pa_status pa_prefix_evictable(const pa_pool *p, int32_t *out, int32_t cap, int32
     *n = p->ev_count;
     int32_t k = 0;
     for (int32_t b = p->ev_head; b >= 0 && k < cap; b = p->ev_next[b]) out[k++] = b;
+    return PA_OK;
+}
+
+static size_t swap_bytes_of(const pa_pool *p, int32_t len) {
+    const size_t nblk = (size_t)((len + p->cfg.block_size - 1) / p->cfg.block_size);
+    return nblk * (size_t)p->cfg.num_layers * 2 * p->block_bytes();
+}
+
+pa_status pa_swap_bytes(const pa_pool *p, int32_t seq_id, size_t *bytes) {
+    if (!p || !bytes) return fail(PA_ERR_INVALID_ARG, "pa_swap_bytes: null argument");
+    auto it = p->seqs.find(seq_id);
+    if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_swap_bytes: unknown sequence");
+    *bytes = swap_bytes_of(p, it->second.len);
+    return PA_OK;
+}
+
+pa_status pa_swap_out(pa_pool *p, int32_t seq_id, void *host_buf, size_t buf_bytes, pa_stream stream) {
+    if (!p) return fail(PA_ERR_INVALID_ARG, "pa_swap_out: null pool");
+    auto it = p->seqs.find(seq_id);
+    if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_swap_out: unknown sequence");
+    pa_pool::Seq &s = it->second;
+    if (s.swapped) return fail(PA_ERR_INVALID_ARG, "pa_swap_out: sequence is already swapped out");
+    if (p->k_pool) {
+        if (!host_buf || buf_bytes < swap_bytes_of(p, s.len))
+            return fail(PA_ERR_INVALID_ARG, "pa_swap_out: host buffer missing or smaller than pa_swap_bytes");
+        pa_status st = pa_internal::swap_copy(p, s.table.data(), (int32_t)s.table.size(), host_buf, true, stream);
+        if (st != PA_OK) return st;
+    }
+    for (int32_t b : s.table)
+        if (drop_ref(p, b)) release(p, b);
+    s.table.clear();
+    s.swapped = true;
+    return PA_OK;
+}
+
+pa_status pa_swap_in(pa_pool *p, int32_t seq_id, const void *host_buf, size_t buf_bytes, pa_stream stream) {
+    if (!p) return fail(PA_ERR_INVALID_ARG, "pa_swap_in: null pool");
+    auto it = p->seqs.find(seq_id);
+    if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_swap_in: unknown sequence");
+    pa_pool::Seq &s = it->second;
+    if (!s.swapped) return fail(PA_ERR_INVALID_ARG, "pa_swap_in: sequence is not swapped out");
+    if (p->k_pool && (!host_buf || buf_bytes < swap_bytes_of(p, s.len)))
+        return fail(PA_ERR_INVALID_ARG, "pa_swap_in: host buffer missing or smaller than pa_swap_bytes");
+    const int32_t n = (s.len + p->cfg.block_size - 1) / p->cfg.block_size;
+    std::vector<int32_t> blocks;
+    std::vector<std::pair<int32_t, uint64_t>> evicted;   // for rollback
+    for (int32_t i = 0; i < n; ++i) {
+        int32_t b;
+        bool ev;
+        uint64_t key;
+        pa_status st = pop_block(p, &b, &ev, &key);
+        if (st != PA_OK) {
+            std::string msg = pa_last_error();
+            for (int32_t j = (int32_t)blocks.size() - 1; j >= 0; --j) {   // undo in reverse
+                const int32_t x = blocks[j];
+                p->refcount[x] = 0;
+                if (evicted[j].first) {
+                    register_key(p, x, evicted[j].second);
+                    ev_push_front(p, x);
+                    --p->cache_evictions;
+                } else {
+                    p->free_stack.push_back(x);
+                }
+            }
+            return fail(st, "pa_swap_in: " + msg + " (no change made)");
+        }
+        blocks.push_back(b);
+        evicted.push_back({ev ? 1 : 0, key});
+    }
+    if (p->k_pool) {
+        pa_status st = pa_internal::swap_copy(p, blocks.data(), n, const_cast<void *>(host_buf), false, stream);
+        if (st != PA_OK) {   // launch failed: give the blocks back
+            for (int32_t j = n - 1; j >= 0; --j) {
+                p->refcount[blocks[j]] = 0;
+                p->free_stack.push_back(blocks[j]);
+            }
+            return st;
+        }
+    }
+    s.table = std::move(blocks);
+    s.swapped = false;
+    note_usage(p);
     return PA_OK;
 }
 

@@ -920,6 +920,40 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p) {
     for (int64_t t = threadIdx.x; t < p.block_chunks; t += blockDim.x) to[t] = from[t];
 }
 
+// ------------------------------------------------------------------ swap copies
+constexpr int kSwapChunk = 256;   // block ids passed by value per launch
+
+struct SwapParams {
+    unsigned char *k_pool;
+    unsigned char *v_pool;
+    unsigned char *host;          // device-visible address of the page-locked host buffer
+    int64_t block_chunks;         // 16-byte chunks of one block (all heads) in one layer
+    int64_t layer_chunks;         // 16-byte chunks of one layer of the pool
+    int32_t num_blocks, first, count, to_host;
+    int32_t blocks[kSwapChunk];
+};
+
+// grid (block in chunk, layer, K|V): one CTA moves one block of one layer of K or V.
+__global__ void __launch_bounds__(256) swap_copy_kernel(const __grid_constant__ SwapParams p) {
+    const int i = blockIdx.x;
+    const int layer = blockIdx.y;
+    const int kv = blockIdx.z;
+    const int blk = p.blocks[i];
+    if ((unsigned)blk >= (unsigned)p.num_blocks) {
+        if (threadIdx.x == 0) raise_error(kErrBadBlock);
+        return;
+    }
+    uint4 *pool = reinterpret_cast<uint4 *>(kv == 0 ? p.k_pool : p.v_pool) + layer * p.layer_chunks +
+                  (int64_t)blk * p.block_chunks;
+    const int64_t layers = gridDim.y;
+    uint4 *host = reinterpret_cast<uint4 *>(p.host) +
+                  (((int64_t)(p.first + i) * layers + layer) * 2 + kv) * p.block_chunks;
+    if (p.to_host)
+        for (int64_t t = threadIdx.x; t < p.block_chunks; t += blockDim.x) host[t] = pool[t];
+    else
+        for (int64_t t = threadIdx.x; t < p.block_chunks; t += blockDim.x) pool[t] = host[t];
+}
+
 // ------------------------------------------------------------------ host dispatch
 pa_status check_launch(const char *what) {
     cudaError_t e = cudaGetLastError();
@@ -1279,3 +1313,39 @@ pa_status pa_device_error(int32_t *code, int32_t clear) {
 }
 
 }  // extern "C"
+
+namespace pa_internal {
+
+pa_status swap_copy(const pa_pool *pool, const int32_t *blocks, int32_t n, void *host_buf, bool to_host,
+                    void *stream) {
+    if (n == 0) return PA_OK;
+    cudaPointerAttributes attr;
+    cudaError_t e = cudaPointerGetAttributes(&attr, host_buf);
+    if (e != cudaSuccess || attr.type != cudaMemoryTypeHost || !attr.devicePointer) {
+        cudaGetLastError();
+        return fail(PA_ERR_INVALID_ARG, "swap: the host buffer must be page-locked host memory the GPU can reach");
+    }
+    if (((uintptr_t)attr.devicePointer & 15) || pool->block_bytes() % 16)
+        return fail(PA_ERR_INVALID_ARG, "swap: host buffer must be 16-byte aligned");
+    if (pool->cfg.num_layers > 65535) return fail(PA_ERR_UNSUPPORTED, "swap: too many layers");
+    SwapParams p;
+    p.k_pool = static_cast<unsigned char *>(pool->k_pool);
+    p.v_pool = static_cast<unsigned char *>(pool->v_pool);
+    p.host = static_cast<unsigned char *>(attr.devicePointer);
+    p.block_chunks = (int64_t)(pool->block_bytes() / 16);
+    p.layer_chunks = (int64_t)(pool->layer_bytes() / 16);
+    p.num_blocks = pool->cfg.num_blocks;
+    p.to_host = to_host ? 1 : 0;
+    for (int32_t first = 0; first < n; first += kSwapChunk) {
+        p.first = first;
+        p.count = n - first < kSwapChunk ? n - first : kSwapChunk;
+        for (int32_t j = 0; j < p.count; ++j) p.blocks[j] = blocks[first + j];
+        swap_copy_kernel<<<dim3(p.count, pool->cfg.num_layers, 2), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+        launch_count.fetch_add(1);
+        pa_status st = check_launch("swap_copy_kernel");
+        if (st != PA_OK) return st;
+    }
+    return PA_OK;
+}
+
+}  // namespace pa_internal

@@ -23,6 +23,7 @@ struct pa_pool {
     struct Seq {
         std::vector<int32_t> table;   // logical block -> physical block
         int32_t len = 0;              // tokens
+        bool swapped = false;         // blocks live in host memory (pa_swap_out)
     };
     std::unordered_map<int32_t, Seq> seqs;
     int32_t next_seq = 0;
@@ -63,4 +64,8 @@ namespace pa_internal {
 pa_status fail(pa_status st, const std::string &msg);
 pa_status ok();
 extern std::atomic<uint64_t> launch_count;
+// Device side of swapping (kernels.cu): copy `blocks` between the pools and a host
+// buffer laid out [block][layer][K, V][Hkv][B][D]; to_host selects the direction.
+pa_status swap_copy(const pa_pool *pool, const int32_t *blocks, int32_t n, void *host_buf, bool to_host,
+                    void *stream);
 }  // namespace pa_internal
