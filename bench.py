@@ -39,9 +39,9 @@ METRIC = "paged decode attention KV-read HBM GB/s (fraction of ~8 TB/s) and deco
 UNIT = "GB/s"
 NOMINAL_HBM_GBS = 8000.0
 WORKLOADS = ("continuous_batch", "large_pool_b16", "large_pool_b32", "worked_example", "prefix_sharing",
-             "shared_prompt")
+             "shared_prompt", "swap")
 DEFAULT_SPLIT = {"continuous_batch": 2048, "large_pool_b16": 2048, "large_pool_b32": 2048,
-                 "worked_example": 128, "prefix_sharing": 1024, "shared_prompt": 2048}
+                 "worked_example": 128, "prefix_sharing": 1024, "shared_prompt": 2048, "swap": 0}
 NSETS = 4           # device input/metadata buffer sets: the host may run this many steps ahead
 
 
@@ -61,7 +61,7 @@ def parse(argv=None):
                     help="shared_prompt workload: share the cached system-prompt blocks at admission")
     a = ap.parse_args(argv)
     if a.steps is None:
-        a.steps = 8 if a.workload.startswith("large_pool") else 64
+        a.steps = 8 if a.workload.startswith("large_pool") or a.workload == "swap" else 64
     if a.split is None:
         a.split = DEFAULT_SPLIT[a.workload]
     return a
@@ -660,8 +660,76 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_swap(args):
+    """Preemption with swap: 64 sequences of the continuous batch (~0.5 GB of cache) moved to
+    page-locked host memory and back, timed with CUDA events, next to a plain pinned
+    cudaMemcpy of the same size (the PCIe roofline of this box)."""
+    import torch
+    import paged_kv_cache_403_b200 as pa
+    from paged_kv_cache_403_b200.engine import PagedCache
+    from paged_kv_cache_403_b200.runners import DeviceGen, prefill
+    from synthetic import workloads as wl
+    torch.cuda.set_device(0)
+    r = wl.continuous_batch(seed=3, steps=1)
+    sh = r["shape"]
+    cache = PagedCache.from_shape(sh, r["order"], "cuda")
+    gen = DeviceGen(r["seed"], sh, "cuda")
+    lens = [int(x) for x in r["schedule"].initial]
+    sids = [cache.add() for _ in lens]
+    prefill(cache, gen, sids, list(range(len(lens))), lens)
+    victims = sids[:64]
+    sizes = [pa.pa_swap_bytes(cache.pool, s) for s in victims]
+    bufs = [torch.empty(n, dtype=torch.uint8).pin_memory() for n in sizes]
+    total = sum(sizes)
+    st = torch.cuda.current_stream()
+
+    def timed(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(st)
+        fn()
+        e1.record(st)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    def out_all():
+        for s, b in zip(victims, bufs):
+            pa.pa_swap_out(cache.pool, s, b)
+
+    def in_all():
+        for s, b in zip(victims, bufs):
+            pa.pa_swap_in(cache.pool, s, b)
+
+    results = {"out": [], "in": []}
+    for rep in range(args.warmup + args.steps):
+        t_out = timed(out_all)
+        t_in = timed(in_all)
+        if rep >= args.warmup:
+            results["out"].append(t_out)
+            results["in"].append(t_in)
+    dev = torch.empty(total, dtype=torch.uint8, device="cuda")
+    host = torch.empty(total, dtype=torch.uint8).pin_memory()
+    d2h = min(timed(lambda: host.copy_(dev, non_blocking=True)) for _ in range(5))
+    h2d = min(timed(lambda: dev.copy_(host, non_blocking=True)) for _ in range(5))
+    gbs = lambda ms: total / (ms * 1e-3) / 1e9  # noqa: E731
+    out_ms, in_ms = float(np.median(results["out"])), float(np.median(results["in"]))
+    line = {"metric": "swap GB/s (device->host and host->device of a sequence's KV blocks)",
+            "value": round(gbs(out_ms + in_ms) * 2, 1), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "dtype": sh.dtype, "data": "synthetic",
+            "config": {"workload": f"swap 64 of 256 continuous-batch sequences, {total / 1e6:.0f} MB of KV"},
+            "swap_out": {"ms": round(out_ms, 3), "GB/s": round(gbs(out_ms), 1)},
+            "swap_in": {"ms": round(in_ms, 3), "GB/s": round(gbs(in_ms), 1)},
+            "roofline": {"bound": "pcie", "d2h_memcpy_GB/s": round(gbs(d2h), 1), "h2d_memcpy_GB/s": round(gbs(h2d), 1),
+                         "frac_out": round(gbs(out_ms) / gbs(d2h), 3), "frac_in": round(gbs(in_ms) / gbs(h2d), 3)},
+            "device_error": pa.pa_device_error()}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.workload == "swap":
+        run_swap(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
