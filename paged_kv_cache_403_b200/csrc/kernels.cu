@@ -791,11 +791,26 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) paged_decode_mma_kernel(con
                 {
                     const int mi = lane >> 3;
                     const int r = j * 16 + (lane & 7) + (mi >> 1) * 8;
+                    // Slots past the sequence end carry weight 0, but their values are
+                    // whatever the pool holds (possibly NaN bit patterns) and 0 * NaN is
+                    // NaN: zero those tokens in the V^T fragments.  Lane (gq, tq) holds
+                    // tokens 2tq, 2tq+1 in a0/a1 and 2tq+8, 2tq+9 in a2/a3.
+                    const int left = L - (tok0 + j * 16);           // valid tokens in this group
+                    uint32_t keep01 = 0xffffffffu, keep89 = 0xffffffffu;
+                    if (left < 16) {
+                        const int t0 = 2 * tq;
+                        keep01 = (t0 < left ? 0x0000ffffu : 0u) | (t0 + 1 < left ? 0xffff0000u : 0u);
+                        keep89 = (t0 + 8 < left ? 0x0000ffffu : 0u) | (t0 + 9 < left ? 0xffff0000u : 0u);
+                    }
 #pragma unroll
                     for (int dm = 0; dm < KD; ++dm) {
                         const int chunk = (dm & 3) * 2 + (mi & 1);
                         uint32_t a[4];
                         ldsm_x4_trans(a, vbase + (dm >> 2) * BOX + r * 128 + ((chunk ^ (r & 7)) << 4));
+                        a[0] &= keep01;
+                        a[1] &= keep01;
+                        a[2] &= keep89;
+                        a[3] &= keep89;
                         M::mma(o[dm], a, bh0, bh1);
                         M::mma(o[dm], a, bl0, bl1);
                     }

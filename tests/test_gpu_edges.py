@@ -42,7 +42,7 @@ class Case:
     """Sequences with given host K/V/q, placed through the library, and the oracle result."""
 
     def __init__(self, lens, B=16, hq=8, hkv=2, d=128, dtype="bf16", order=None, nb=None, seed=0,
-                 kv_scale=1.0, q_scale=1.0, k_override=None):
+                 kv_scale=1.0, q_scale=1.0, k_override=None, fill=None):
         self.lens, self.B, self.hq, self.hkv, self.d, self.dtype = list(lens), B, hq, hkv, d, dtype
         nb = nb or sum(-(-L // B) for L in lens) + 8
         rng = np.random.default_rng(seed)
@@ -54,6 +54,9 @@ class Case:
                   for L in lens]
         self.q = sv.narrow((rng.standard_normal((len(lens), hq, d)) * q_scale).astype(np.float32), dtype)
         self.cache = PagedCache(1, nb, B, hkv, d, dtype, order)
+        if fill is not None:                 # what unused slots hold before anything is written
+            self.cache.k_pool.fill_(fill)
+            self.cache.v_pool.fill_(fill)
         self.sids = [self.cache.add() for _ in lens]
         slots, _ = self.cache.reserve(self.sids, self.lens)
         kk = np.concatenate(self.k) if lens else np.zeros((0, hkv, d))
@@ -162,6 +165,21 @@ def test_peaky_and_increasing_scores():
         check_close(c.run(split), ref, "f32", "f32", f"peaky split {split}")
     c2 = Case([1000, 257], hq=8, hkv=2, q_scale=25.0)
     check_close(c2.run(0), c2.oracle(), "f32", "bf16", "large q")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("B", [16, 32])
+def test_unused_slots_holding_nan_do_not_leak(dtype, B):
+    """Pools whose unused slots hold NaN (memory never written): every tail block has
+    NaN rows past the sequence end; outputs must stay finite and match the oracle."""
+    lens = [1, 5, 17, 31, 33, 100, 511]
+    c = Case(lens, B=B, dtype=dtype, fill=float("nan"),
+             order=list(np.random.default_rng(8).permutation(sum(-(-L // B) for L in lens) + 8)))
+    ref = c.oracle()
+    for split in (0, 2 * B):
+        out = c.run(split)
+        assert np.isfinite(out).all()
+        check_close(out, ref, "f32", dtype, f"nan pool split {split}")
 
 
 def test_empty_batch_launches_nothing():
