@@ -38,6 +38,12 @@ def lib():
             ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
             ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_void_p,
             ctypes.c_int]
+        L.oracle_paged_prefill.restype = ctypes.c_int
+        L.oracle_paged_prefill.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_int]
         L.oracle_widen.restype = None
         L.oracle_widen.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p]
         L.oracle_max_threads.restype = ctypes.c_int
@@ -79,6 +85,31 @@ def paged_decode(k_layer: np.ndarray, v_layer: np.ndarray, dtype: str, tables, l
                                    float(scale), _ptr(out), int(n_threads))
     if rc != 0:
         raise ValueError("oracle_paged_decode rejected its arguments")
+    return out
+
+
+def paged_prefill(k_layer: np.ndarray, v_layer: np.ndarray, dtype: str, tables, lens, q_start,
+                  q: np.ndarray, scale: float, n_threads: int = 0) -> np.ndarray:
+    """fp64 causal chunked-prefill attention over the paged cache.
+
+    q_start [n+1]: sequence s owns query rows q_start[s]..q_start[s+1]-1, the last
+    tokens of its length lens[s].  Returns [total_q][num_q_heads][head_dim] float64.
+    """
+    k = np.ascontiguousarray(k_layer)
+    v = np.ascontiguousarray(v_layer)
+    nb, hkv, bs, d = k.shape
+    t = np.ascontiguousarray(tables, dtype=np.int32)
+    ln = np.ascontiguousarray(lens, dtype=np.int32)
+    qs = np.ascontiguousarray(q_start, dtype=np.int32)
+    qq = np.ascontiguousarray(q)
+    rows, hq, dq = qq.shape
+    assert dq == d and qs[-1] == rows and t.shape[0] == ln.shape[0] == qs.shape[0] - 1
+    out = np.empty((rows, hq, d), np.float64)
+    rc = lib().oracle_paged_prefill(_ptr(k), _ptr(v), _CODES[dtype], nb, bs, hkv, d, _ptr(t), t.shape[1],
+                                    _ptr(ln), _ptr(qs), ln.shape[0], _ptr(qq), hq, float(scale), _ptr(out),
+                                    int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_paged_prefill rejected its arguments")
     return out
 
 

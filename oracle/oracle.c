@@ -165,6 +165,94 @@ int oracle_paged_decode(const void *k_pool, const void *v_pool, int dtype,
     return 0;
 }
 
+/*
+ * Paged chunked-prefill attention (causal), the same definition applied to every
+ * query of a prompt chunk: "What problem does PagedAttention solve, and what is
+ * continuous batching?", sections "Why the KV cache becomes the problem" (prefill
+ * is the pass over the prompt) and "The prefill and decode phases need careful
+ * scheduling" (chunked prefill breaks a long prompt into pieces).  Reading: the
+ * chunk's keys and values are already in the cache, the chunk is the last C_s
+ * tokens of sequence s, and the query at absolute position p attends to keys 0..p.
+ *   q     : [total_q][num_q_heads][head_dim]; sequence s owns rows
+ *           q_start[s] .. q_start[s+1]-1 (C_s rows, C_s <= lens[s])
+ *   out   : same shape, double
+ * Returns 0, or -1 for an invalid argument (nothing written then).
+ */
+int oracle_paged_prefill(const void *k_pool, const void *v_pool, int dtype,
+                         int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
+                         const int32_t *tables, int max_blocks, const int32_t *lens,
+                         const int32_t *q_start, int n_seqs, const void *q, int num_q_heads,
+                         double scale, double *out, int n_threads)
+{
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || block_size <= 0 || head_dim <= 0)
+        return -1;
+    for (int s = 0; s < n_seqs; ++s) {
+        int L = lens[s], C = q_start[s + 1] - q_start[s];
+        if (L < 1 || C < 0 || C > L || (L + block_size - 1) / block_size > max_blocks)
+            return -1;
+        for (int b = 0; b < (L + block_size - 1) / block_size; ++b) {
+            int32_t blk = tables[(size_t)s * max_blocks + b];
+            if (blk < 0 || blk >= num_blocks)
+                return -1;
+        }
+    }
+    const int group = num_q_heads / num_kv_heads;
+    const long total_rows = q_start[n_seqs];
+#ifdef _OPENMP
+    const int nt = n_threads > 0 ? n_threads : omp_get_num_procs();
+#else
+    (void)n_threads;
+#endif
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (long rh = 0; rh < total_rows * num_q_heads; ++rh) {
+        const long row = rh / num_q_heads;
+        const int h = (int)(rh % num_q_heads);
+        const int g = h / group;
+        int s = 0;
+        while (q_start[s + 1] <= row)
+            ++s;
+        const int L = lens[s];
+        const int C = q_start[s + 1] - q_start[s];
+        const int p = L - C + (int)(row - q_start[s]);      /* absolute position of this query */
+        const int nkeys = p + 1;                              /* causal: keys 0..p */
+        double *z = malloc(sizeof(double) * (size_t)nkeys);
+        double *qh = malloc(sizeof(double) * (size_t)head_dim);
+        for (int i = 0; i < head_dim; ++i)
+            qh[i] = load_elem(q, dtype, ((size_t)row * num_q_heads + h) * head_dim + i);
+        double zmax = -INFINITY;
+        for (int j = 0; j < nkeys; ++j) {
+            int32_t blk = tables[(size_t)s * max_blocks + j / block_size];
+            size_t base = (((size_t)blk * num_kv_heads + g) * block_size + j % block_size) * head_dim;
+            double acc = 0.0;
+            for (int i = 0; i < head_dim; ++i)
+                acc += qh[i] * load_elem(k_pool, dtype, base + i);
+            z[j] = scale * acc;
+            if (z[j] > zmax)
+                zmax = z[j];
+        }
+        double denom = 0.0;
+        for (int j = 0; j < nkeys; ++j) {
+            z[j] = exp(z[j] - zmax);
+            denom += z[j];
+        }
+        double *o = out + ((size_t)row * num_q_heads + h) * head_dim;
+        for (int i = 0; i < head_dim; ++i)
+            o[i] = 0.0;
+        for (int j = 0; j < nkeys; ++j) {
+            int32_t blk = tables[(size_t)s * max_blocks + j / block_size];
+            size_t base = (((size_t)blk * num_kv_heads + g) * block_size + j % block_size) * head_dim;
+            for (int i = 0; i < head_dim; ++i)
+                o[i] += z[j] * load_elem(v_pool, dtype, base + i);
+        }
+        for (int i = 0; i < head_dim; ++i)
+            o[i] /= denom;
+        free(z);
+        free(qh);
+    }
+    return 0;
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP
