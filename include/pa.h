@@ -283,6 +283,23 @@ pa_status pa_decode_attention_static(pa_pool *pool, int32_t layer, const void *q
                                      int32_t n_seqs, int32_t num_q_heads, float scale,
                                      int32_t split_tokens, pa_stream stream);
 
+/* Paged chunked-prefill attention (causal) on the tensor cores ([P1] "Why the KV
+ * cache becomes the problem": prefill is the compute-heavy pass over the prompt;
+ * "The prefill and decode phases need careful scheduling": long prompts are split
+ * into chunks).  For sequence s the chunk is its last C_s = q_start_dev[s+1] -
+ * q_start_dev[s] tokens, already appended to the cache (seq_lens_dev[s] counts them);
+ * query row q_start_dev[s] + i sits at position L_s - C_s + i and attends to keys
+ * 0 .. L_s - C_s + i through the block table:
+ *   out[r][h] = sum_{j <= pos(r)} softmax_j(scale * q[r][h] . K_s[j]) V_s[j].
+ * q [total][num_q_heads][128] in the pool dtype (fp16 or bf16), out the same shape in
+ * out_dtype (PA_F32 or the pool dtype), q_start_dev int32 [n_seqs + 1] ascending,
+ * max_q_len >= every C_s.  head_dim 128, block_size 16 or 32, num_q_heads /
+ * num_kv_heads in {1, 2, 4, 8}; fp32 caches -> PA_ERR_UNSUPPORTED. */
+pa_status pa_prefill_attention(pa_pool *pool, int32_t layer, const void *q, void *out, pa_dtype out_dtype,
+                               const int32_t *block_tables_dev, int32_t max_blocks,
+                               const int32_t *seq_lens_dev, const int32_t *q_start_dev, int32_t n_seqs,
+                               int32_t max_q_len, int32_t num_q_heads, float scale, pa_stream stream);
+
 /* ------------------------------------------------------------------ diagnostics */
 
 /* Device error bits recorded by kernels since the last clear (synchronises the

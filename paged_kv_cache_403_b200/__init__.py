@@ -275,6 +275,16 @@ def pa_decode_attention(pool, layer: int, q, out, block_tables_dev, seq_lens_dev
                                       _stream(stream)))
 
 
+def pa_prefill_attention(pool, layer: int, q, out, block_tables_dev, seq_lens_dev, q_start_dev,
+                         max_q_len: int, scale: float, stream=None) -> None:
+    """Causal chunked-prefill attention: q / out [total][Hq][128], q_start [n + 1] (CUDA tensors)."""
+    n = seq_lens_dev.shape[0]
+    _check(_lib().pa_prefill_attention(pool, layer, _dev_ptr(q), _dev_ptr(out), _dtype_code(out.dtype),
+                                       _dev_ptr(block_tables_dev), block_tables_dev.shape[1],
+                                       _dev_ptr(seq_lens_dev), _dev_ptr(q_start_dev), n, max_q_len, q.shape[1],
+                                       float(scale), _stream(stream)))
+
+
 PA_STATIC_WORKSPACE_BYTES = 16 << 20
 
 

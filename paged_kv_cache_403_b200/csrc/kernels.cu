@@ -878,6 +878,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) paged_decode_mma_kernel(con
     }
 }
 
+#include "prefill.cuh"
+
 // ------------------------------------------------------------------ append / copy
 struct AppendParams {
     unsigned char *k_layer;
@@ -1090,6 +1092,19 @@ pa_status ensure_tensor_maps(pa_pool *pool) {
     return PA_OK;
 }
 
+// One shared-memory flag per kernel instantiation (the flag must not be shared between
+// kernels of the same pointer type).
+template <typename T, int B>
+pa_status launch_prefill(const prefill::Params &p, dim3 grid, cudaStream_t stream) {
+    auto kernel = prefill::paged_prefill_kernel<T, B>;
+    static bool smem_set[64] = {};
+    pa_status st = ensure_smem(kernel, prefill::kSmemBytes, smem_set);
+    if (st != PA_OK) return st;
+    kernel<<<grid, prefill::kThreads, prefill::kSmemBytes, stream>>>(p);
+    pa_internal::launch_count.fetch_add(1);
+    return check_launch("paged_prefill_kernel");
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 }  // namespace
@@ -1236,6 +1251,62 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
     p.scale_log2 = scale_log2;
     if (c.dtype == PA_BF16) return dispatch_mma<__nv_bfloat16>(p, r, n_seqs, c.block_size, c.head_dim, st);
     return dispatch_mma<__half>(p, r, n_seqs, c.block_size, c.head_dim, st);
+}
+
+pa_status pa_prefill_attention(pa_pool *pool, int32_t layer, const void *q, void *out, pa_dtype out_dtype,
+                               const int32_t *block_tables_dev, int32_t max_blocks, const int32_t *seq_lens_dev,
+                               const int32_t *q_start_dev, int32_t n_seqs, int32_t max_q_len, int32_t num_q_heads,
+                               float scale, pa_stream stream) {
+    if (!pool || !pool->k_pool) return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: pool has no device memory");
+    const pa_pool_config &c = pool->cfg;
+    if (layer < 0 || layer >= c.num_layers) return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: layer out of range");
+    if (n_seqs < 0 || max_blocks < 1 || max_q_len < 0)
+        return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: bad n_seqs / max_blocks / max_q_len");
+    if (n_seqs == 0 || max_q_len == 0) return PA_OK;
+    if (!q || !out || !block_tables_dev || !seq_lens_dev || !q_start_dev)
+        return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: null device pointer");
+    if (!aligned16(q) || !aligned16(out) || ((uintptr_t)block_tables_dev & 3) || ((uintptr_t)seq_lens_dev & 3) ||
+        ((uintptr_t)q_start_dev & 3))
+        return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: misaligned pointer");
+    if (c.dtype == PA_F32)
+        return fail(PA_ERR_UNSUPPORTED, "pa_prefill_attention: the tensor-core path takes fp16 / bf16 caches");
+    if (c.head_dim != 128 || (c.block_size != 16 && c.block_size != 32))
+        return fail(PA_ERR_UNSUPPORTED, "pa_prefill_attention: head_dim 128 and block_size 16 or 32 only");
+    if (out_dtype != PA_F32 && out_dtype != c.dtype)
+        return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: out_dtype must be PA_F32 or the pool dtype");
+    if (num_q_heads < 1 || num_q_heads % c.num_kv_heads != 0)
+        return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: num_q_heads must be a multiple of num_kv_heads");
+    const int group = num_q_heads / c.num_kv_heads;
+    if (group != 1 && group != 2 && group != 4 && group != 8)
+        return fail(PA_ERR_UNSUPPORTED, "pa_prefill_attention: query heads per KV head must be 1, 2, 4 or 8");
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: scale must be finite");
+    const int64_t tiles = ((int64_t)max_q_len * group + prefill::kRows - 1) / prefill::kRows;
+    if (tiles > INT32_MAX || c.num_kv_heads > 65535 || n_seqs > 65535)
+        return fail(PA_ERR_UNSUPPORTED, "pa_prefill_attention: grid too large");
+    pa_status st = ensure_tensor_maps(pool);
+    if (st != PA_OK) return st;
+    prefill::Params p;
+    p.tmap_k = pool->tmap_k;
+    p.tmap_v = pool->tmap_v;
+    p.q = q;
+    p.out = out;
+    p.tables = block_tables_dev;
+    p.lens = seq_lens_dev;
+    p.q_start = q_start_dev;
+    p.max_blocks = max_blocks;
+    p.num_blocks = c.num_blocks;
+    p.num_kv_heads = c.num_kv_heads;
+    p.num_q_heads = num_q_heads;
+    p.layer = layer;
+    p.block_size = c.block_size;
+    p.out_f32 = out_dtype == PA_F32;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    const dim3 grid((unsigned)tiles, c.num_kv_heads, n_seqs);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (c.dtype == PA_BF16)
+        return c.block_size == 16 ? launch_prefill<__nv_bfloat16, 16>(p, grid, cs)
+                                  : launch_prefill<__nv_bfloat16, 32>(p, grid, cs);
+    return c.block_size == 16 ? launch_prefill<__half, 16>(p, grid, cs) : launch_prefill<__half, 32>(p, grid, cs);
 }
 
 pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const void *v_new,

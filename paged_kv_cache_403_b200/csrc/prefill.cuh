@@ -1,0 +1,410 @@
+// Paged chunked-prefill attention on the 5th-generation tensor cores (tcgen05, TMEM).
+// Included by kernels.cu (shares its device error word, mbarrier and TMA helpers).
+//
+// "What problem does PagedAttention solve, and what is continuous batching?": prefill
+// is the compute-heavy pass over the prompt ("Why the KV cache becomes the problem")
+// and long prompts are broken into chunks ("The prefill and decode phases need careful
+// scheduling").  A chunk is the last C tokens of a sequence whose keys and values are
+// already in the paged cache; query i of the chunk (absolute position L - C + i)
+// attends to keys 0 .. L - C + i, read through the block table.
+//
+// One CTA per (128-row query tile, KV head, sequence).  Rows are (token, query head of
+// the GQA group) pairs, row = token * G + head, so every query head of the group
+// shares each key/value tile.  Per 64-key tile (64 / block_size blocks):
+//   TMA (2-D tensor loads, 128-byte swizzle) of K and V into a 2-stage ring;
+//   S = Q K^T        tcgen05.mma kind::f16, M=128, N=64, K=head_dim, D in TMEM;
+//   softmax          each thread owns one row = one TMEM lane: tcgen05.ld of its 64
+//                    scores, causal / length mask by select, base-2 online softmax
+//                    with a lazily moved maximum (rescales O in TMEM only when a score
+//                    passes the running maximum by 2^8), P split into a 16-bit high
+//                    part and the 16-bit rounding of the remainder, both written to
+//                    shared memory in the K-major swizzled layout;
+//   O += P V         tcgen05.mma kind::f16, M=128, N=head_dim, K=64, once with the
+//                    high part and once with the remainder (about 16 bits of each
+//                    weight survive), V read as an MN-major operand straight from the
+//                    TMA tile.
+// Key rows past the sequence end are zeroed in shared memory before P V (their weight
+// is 0, but 0 * NaN would not be).  Version 1 runs S, softmax and P V one after the
+// other; the TMA ring prefetches the next tile meanwhile.
+namespace prefill {
+
+constexpr int kRows = 128;           // MMA M: query rows of a tile
+constexpr int kKeys = 64;            // keys per tile
+constexpr int kThreads = 128;        // one thread per row / TMEM lane
+constexpr int kD = 128;              // head_dim
+constexpr uint32_t kTmemCols = 256;  // O in [0, 128), S in [128, 192)
+constexpr uint32_t kOCol = 0, kSCol = 128;
+constexpr int kQBytes = kRows * kD * 2;         // 32 KB: [2 halves][128 rows][128 B]
+constexpr int kKVBytes = kKeys * kD * 2;        // 16 KB: [2 halves][64 rows][128 B]
+constexpr int kPBytes = kRows * kKeys * 2;      // 16 KB: [128 rows][128 B], high and low parts
+constexpr int kStages = 2;
+constexpr int kSmemBytes = 1024 + kQBytes + kStages * 2 * kKVBytes + 2 * kPBytes + 64;
+
+// --- tcgen05 wrappers --------------------------------------------------------------
+// Shared-memory matrix descriptor, 128-byte swizzle: start address, leading and stride
+// byte offsets in 16-byte units, descriptor version 1, layout code 2 (SWIZZLE_128B).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, A/B format (0 = f16, 1 = bf16),
+// A/B major-ness (0 = K-major, 1 = MN-major), N / 8 and M / 16.
+__host__ __device__ constexpr uint32_t instr_desc(uint32_t fmt, uint32_t m, uint32_t n, uint32_t a_mn,
+                                                  uint32_t b_mn) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | (a_mn << 15) | (b_mn << 16) | ((n >> 3) << 17) |
+           ((m >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_before_sync() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// generic-proxy shared-memory writes become visible to the tensor core (async proxy)
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Bounded wait polled by every thread; a thread that gives up sets the abort flag so
+// the others stop polling.  Callers combine the results with __syncthreads_and, so
+// the whole CTA takes the same branch.
+__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            raise_error(kErrTimeout);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+template <typename T>
+struct Fmt;
+template <>
+struct Fmt<__half> {
+    static constexpr uint32_t code = 0;
+};
+template <>
+struct Fmt<__nv_bfloat16> {
+    static constexpr uint32_t code = 1;
+};
+
+struct Params {
+    CUtensorMap tmap_k;
+    CUtensorMap tmap_v;
+    const void *q;              // [total_q][Hq][D]
+    void *out;                  // [total_q][Hq][D]
+    const int32_t *tables;      // [n][max_blocks]
+    const int32_t *lens;        // [n] total tokens (context + chunk)
+    const int32_t *q_start;     // [n + 1]
+    int32_t max_blocks, num_blocks, num_kv_heads, num_q_heads, layer, block_size, out_f32;
+    float scale_log2;
+};
+
+template <typename T, int B>
+__global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid_constant__ Params p) {
+    constexpr int BLOCKS_PER_TILE = kKeys / B;
+    constexpr uint32_t IDESC_S = instr_desc(Fmt<T>::code, kRows, kKeys, 0, 0);
+    constexpr uint32_t IDESC_O = instr_desc(Fmt<T>::code, kRows, kD, 0, 1);
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+    unsigned char *sQ = smem;
+    unsigned char *sK = sQ + kQBytes;                    // stage st: sK + st * 2 * kKVBytes
+    unsigned char *sP = sK + kStages * 2 * kKVBytes;          // high part; low part follows
+    uint64_t *full = reinterpret_cast<uint64_t *>(sP + 2 * kPBytes);   // [kStages]
+    uint64_t *mma_bar = full + kStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int s = blockIdx.z;
+    const int g = blockIdx.y;
+    const int qt = blockIdx.x;
+    const int group = p.num_q_heads / p.num_kv_heads;
+    const int tokens_per_tile = kRows / group;
+    const int q0 = p.q_start[s];
+    const int C = p.q_start[s + 1] - q0;
+    const int t0 = qt * tokens_per_tile;
+    if (t0 >= C) return;
+    int L = p.lens[s];
+    const int nblk = (L + B - 1) / B;
+    if (L < 1 || C > L || nblk > p.max_blocks) {
+        if (threadIdx.x == 0) raise_error(kErrBadLen);
+        return;
+    }
+    const int P0 = L - C;                                  // position of the chunk's first token
+    const int t_last = min(C, t0 + tokens_per_tile) - 1;
+    const int n_tiles = (P0 + t_last) / kKeys + 1;         // keys 0 .. P0 + t_last
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int32_t *trow = p.tables + (size_t)s * p.max_blocks;
+
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) mbar_init(&full[i], 1);
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0) {   // TMEM: one warp allocates (and later frees) for the CTA
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+
+    // K/V tile loads (thread 0): blocks past the sequence end load the first block
+    // instead (finite data; masked and zeroed before use).
+    auto issue_tile = [&](int j) {
+        const int st = j % kStages;
+        unsigned char *k_dst = sK + st * 2 * kKVBytes;
+        unsigned char *v_dst = k_dst + kKVBytes;
+        mbar_arrive_expect_tx(&full[st], 2 * kKVBytes);
+        for (int b = 0; b < BLOCKS_PER_TILE; ++b) {
+            const int lb = j * BLOCKS_PER_TILE + b;
+            int blk = trow[lb < nblk ? lb : 0];
+            if ((unsigned)blk >= (unsigned)p.num_blocks) {
+                raise_error(kErrBadBlock);
+                blk = 0;
+            }
+            const int row = ((p.layer * p.num_blocks + blk) * p.num_kv_heads + g) * B;
+            for (int h = 0; h < 2; ++h) {
+                tma_load_2d(k_dst + h * (kKVBytes / 2) + b * B * 128, &p.tmap_k, h * 64, row, &full[st]);
+                tma_load_2d(v_dst + h * (kKVBytes / 2) + b * B * 128, &p.tmap_v, h * 64, row, &full[st]);
+            }
+        }
+    };
+
+    // Q tile: row r = token * G + head; rows past the chunk are zero
+    const int my_t = t0 + tid / group;
+    const int my_h = g * group + tid % group;
+    const bool row_valid = my_t < C;
+    {
+        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.q) +
+                                                            ((size_t)(q0 + (row_valid ? my_t : 0)) * p.num_q_heads + my_h) * kD);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const uint4 v = row_valid ? src[c] : make_uint4(0, 0, 0, 0);
+            const int half = c >> 3, cc = c & 7;
+            *reinterpret_cast<uint4 *>(sQ + half * (kQBytes / 2) + tid * 128 + ((cc ^ (tid & 7)) << 4)) = v;
+        }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        issue_tile(0);
+        if (n_tiles > 1) issue_tile(1);
+    }
+
+    const int kmax = row_valid ? P0 + my_t : -1;            // last key this row may see
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float sl = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    const uint32_t qaddr = smem_addr(sQ), paddr = smem_addr(sP);
+    bool ok = true;
+
+    for (int j = 0; j < n_tiles && ok; ++j) {
+        const int st = j % kStages;
+        unsigned char *k_st = sK + st * 2 * kKVBytes;
+        unsigned char *v_st = k_st + kKVBytes;
+        ok = __syncthreads_and(wait_all(&full[st], (j / kStages) & 1, abort_flag));
+        if (!ok) break;
+        // keys past the sequence end: zero their V rows (whole 128-byte rows, both halves)
+        const int first_bad = L - j * kKeys;
+        if (first_bad < kKeys) {
+            const int row = tid >> 1, half = tid & 1;
+            if (row >= first_bad) {
+                uint4 *dst = reinterpret_cast<uint4 *>(v_st + half * (kKVBytes / 2) + row * 128);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async();
+        }
+        fence_before_sync();
+        __syncthreads();
+        // S = Q K^T
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t kaddr = smem_addr(k_st);
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+                const uint64_t a = smem_desc(qaddr + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
+                const uint64_t b = smem_desc(kaddr + (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32, 16, 1024);
+                umma(tmem + kSCol, a, b, IDESC_S, kk > 0);
+            }
+            umma_commit(mma_bar);
+        }
+        ok = __syncthreads_and(wait_all(mma_bar, 0, abort_flag));
+        if (!ok) break;
+        fence_after_sync();
+        uint32_t sv[64];
+        {
+            uint32_t a[32], b[32];
+            tmem_ld32(tmem + lane_base + kSCol, a);
+            tmem_ld32(tmem + lane_base + kSCol + 32, b);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                sv[c] = a[c];
+                sv[32 + c] = b[c];
+            }
+        }
+        // mask, scale, running maximum
+        const int key0 = j * kKeys;
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+            const float x = (key0 + c <= kmax && key0 + c < L) ? __uint_as_float(sv[c]) * sl : -INFINITY;
+            sv[c] = __float_as_uint(x);
+            tmax = fmaxf(tmax, x);
+        }
+        if (tmax > m + kRescaleThreshold) {
+            const float f = ex2(m - tmax);     // 0 while nothing has been accumulated
+            if (j > 0) {                       // O holds earlier tiles: scale this row in TMEM
+#pragma unroll
+                for (int c0 = 0; c0 < kD; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_base + kOCol + c0, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+                    tmem_st32(tmem + lane_base + kOCol + c0, o);
+                }
+                tmem_wait_st();
+            }
+            l *= f;
+            m = tmax;
+        }
+        // P as high + low 16-bit parts (K-major swizzled) and the row sum
+        const bool any = m != -INFINITY;
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+            uint32_t w[4], r[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float x0 = __uint_as_float(sv[c8 * 8 + 2 * e]);
+                const float x1 = __uint_as_float(sv[c8 * 8 + 2 * e + 1]);
+                const float p0 = any ? ex2(x0 - m) : 0.f;
+                const float p1 = any ? ex2(x1 - m) : 0.f;
+                w[e] = Mma<T>::pack(p0, p1);
+                r[e] = Mma<T>::pack(p0 - Mma<T>::low(w[e]), p1 - Mma<T>::high(w[e]));
+                l += p0 + p1;
+            }
+            const int off = tid * 128 + ((c8 ^ (tid & 7)) << 4);
+            *reinterpret_cast<uint4 *>(sP + off) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4 *>(sP + kPBytes + off) = make_uint4(r[0], r[1], r[2], r[3]);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // O += P V
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t vaddr = smem_addr(v_st);
+#pragma unroll
+            for (int kk = 0; kk < kKeys / 16; ++kk) {
+                const uint64_t b = smem_desc(vaddr + kk * 16 * 128, kKVBytes / 2, 1024);
+                umma(tmem + kOCol, smem_desc(paddr + kk * 32, 16, 1024), b, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+                umma(tmem + kOCol, smem_desc(paddr + kPBytes + kk * 32, 16, 1024), b, IDESC_O, 1u);
+            }
+            umma_commit(mma_bar);
+        }
+        ok = __syncthreads_and(wait_all(mma_bar, 1, abort_flag));
+        if (!ok) break;
+        fence_after_sync();
+        if (tid == 0 && j + kStages < n_tiles) issue_tile(j + kStages);
+    }
+
+    if (ok) {
+        // O / l for this row
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const size_t orow = ((size_t)(q0 + my_t) * p.num_q_heads + my_h) * kD;
+#pragma unroll
+        for (int c0 = 0; c0 < kD; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_base + kOCol + c0, o);
+            tmem_wait_ld();
+            if (row_valid) {
+                if (p.out_f32) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + orow + c0);
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4)
+                        dst[c / 4] = make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
+                                                 __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+                } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<T *>(p.out) + orow + c0);
+#pragma unroll
+                    for (int c = 0; c < 32; c += 8) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            w[e] = Mma<T>::pack(__uint_as_float(o[c + 2 * e]) * inv,
+                                                __uint_as_float(o[c + 2 * e + 1]) * inv);
+                        dst[c / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace prefill
