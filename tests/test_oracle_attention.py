@@ -214,11 +214,15 @@ def test_rejects_invalid_tables():
 
 # ---------------------------------------------------------------- planted mistakes
 MUTANTS = {
-    "gqa_modulo": ("const int g = h / group;", "const int g = h % num_kv_heads;"),
-    "gather_swapped": ("j / block_size];", "j % block_size];"),
-    "row_offset": ("+ j % block_size) * head_dim;", "+ j / block_size) * head_dim;"),
-    "no_scale": ("z[j] = scale * acc;", "z[j] = acc;"),
-    "no_max_shift": ("z[j] = exp(z[j] - zmax);", "z[j] = exp(z[j]);"),
+    "gqa_modulo": ("const int g = h / group;\n        const int L = lens[s];",
+                   "const int g = h % num_kv_heads;\n        const int L = lens[s];"),
+    "gather_swapped": ("j / block_size];\n            size_t row", "j % block_size];\n            size_t row"),
+    "row_offset": ("size_t row = (((size_t)blk * num_kv_heads + g) * block_size + j % block_size) * head_dim;",
+                   "size_t row = (((size_t)blk * num_kv_heads + g) * block_size + j / block_size) * head_dim;"),
+    "no_scale": ("acc += qh[i] * K[(size_t)j * head_dim + i];\n            z[j] = scale * acc;",
+                 "acc += qh[i] * K[(size_t)j * head_dim + i];\n            z[j] = acc;"),
+    "no_max_shift": ("for (int j = 0; j < L; ++j) {\n            z[j] = exp(z[j] - zmax);",
+                     "for (int j = 0; j < L; ++j) {\n            z[j] = exp(z[j]);"),
     "k_transposed": ("acc += qh[i] * K[(size_t)j * head_dim + i];",
                      "acc += qh[i] * K[(size_t)i * head_dim + j % head_dim];"),
     "v_for_k": ("K[(size_t)j * head_dim + i] = load_elem(k_pool", "K[(size_t)j * head_dim + i] = load_elem(v_pool"),
@@ -229,7 +233,7 @@ MUTANTS = {
 
 def _compile_mutant(name):
     src = open(ORACLE_C).read()
-    old, new = MUTANTS[name]
+    old, new = (x.replace("\\n", "\n") for x in MUTANTS[name])
     assert src.count(old) == 1, name
     tmpd = tempfile.mkdtemp()
     c = os.path.join(tmpd, "m.c")
