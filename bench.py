@@ -39,9 +39,9 @@ METRIC = "paged decode attention KV-read HBM GB/s (fraction of ~8 TB/s) and deco
 UNIT = "GB/s"
 NOMINAL_HBM_GBS = 8000.0
 WORKLOADS = ("continuous_batch", "large_pool_b16", "large_pool_b32", "worked_example", "prefix_sharing",
-             "shared_prompt", "swap")
+             "shared_prompt", "swap", "prefill")
 DEFAULT_SPLIT = {"continuous_batch": 2048, "large_pool_b16": 2048, "large_pool_b32": 2048,
-                 "worked_example": 128, "prefix_sharing": 1024, "shared_prompt": 2048, "swap": 0}
+                 "worked_example": 128, "prefix_sharing": 1024, "shared_prompt": 2048, "swap": 0, "prefill": 0}
 NSETS = 4           # device input/metadata buffer sets: the host may run this many steps ahead
 
 
@@ -61,7 +61,7 @@ def parse(argv=None):
                     help="shared_prompt workload: share the cached system-prompt blocks at admission")
     a = ap.parse_args(argv)
     if a.steps is None:
-        a.steps = 8 if a.workload.startswith("large_pool") or a.workload == "swap" else 64
+        a.steps = 8 if a.workload.startswith("large_pool") or a.workload in ("swap", "prefill") else 64
     if a.split is None:
         a.split = DEFAULT_SPLIT[a.workload]
     return a
@@ -725,10 +725,123 @@ def run_swap(args):
     print(json.dumps(line), flush=True)
 
 
+def prefill_setup(torch, recipe, device="cuda"):
+    """Cache holding every sequence's tokens, the chunk queries and the launch metadata."""
+    from paged_kv_cache_403_b200.engine import PagedCache
+    from paged_kv_cache_403_b200.runners import DeviceGen, prefill
+    sh = recipe["shape"]
+    cache = PagedCache.from_shape(sh, recipe["order"], device)
+    gen = DeviceGen(recipe["seed"], sh, device)
+    lens = [int(x) for x in recipe["lens"]]
+    chunks = [int(x) for x in recipe["chunks"]]
+    sids = [cache.add() for _ in lens]
+    prefill(cache, gen, sids, list(range(len(lens))), lens)
+    uids = np.concatenate([np.full(c, s) for s, c in enumerate(chunks)])
+    pos = np.concatenate([np.arange(L - c, L) for L, c in zip(lens, chunks)])
+    q = gen.q(0, uids, pos)
+    max_blocks = max(-(-L // sh.block_size) for L in lens)
+    tables, ln = cache.tables(sids, max_blocks)
+    q_start = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    flops = sum(4.0 * (L - c + i + 1) * sh.num_q_heads * sh.head_dim for L, c in zip(lens, chunks) for i in range(c))
+    return dict(cache=cache, q=q, tables=torch.from_numpy(tables).to(device), lens=torch.from_numpy(ln).to(device),
+                q_start=torch.from_numpy(q_start).to(device), max_q=max(chunks), flops=flops, rows=int(q_start[-1]),
+                lens_list=lens, chunks=chunks, uids=uids, pos=pos, tables_np=tables)
+
+
+def run_prefill(args):
+    """Chunked-prefill attention (tcgen05) on the synthetic chunked-prefill workload."""
+    import torch
+    import paged_kv_cache_403_b200 as pa
+    from synthetic import workloads as wl
+    torch.cuda.set_device(0)
+    r = wl.chunked_prefill()
+    sh = r["shape"]
+    c = prefill_setup(torch, r)
+    out = torch.empty((c["rows"], sh.num_q_heads, sh.head_dim), dtype=torch.bfloat16, device="cuda")
+    st = torch.cuda.current_stream()
+    scale = 1.0 / math.sqrt(sh.head_dim)
+
+    def call():
+        pa.pa_prefill_attention(c["cache"].pool, 0, c["q"], out, c["tables"], c["lens"], c["q_start"], c["max_q"],
+                                scale)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    lc0 = pa.pa_launch_count()
+    evs = []
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(st)
+    for _ in range(args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        call()
+        b.record(st)
+        evs.append((a, b))
+    t1.record(st)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    kern_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    peaks = {}
+    pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk_path):
+        peaks = json.load(open(pk_path))
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    achieved = c["flops"] / (kern_ms * 1e-3) / 1e12
+    line = {"metric": "paged chunked-prefill attention TFLOP/s and prefill tokens/s", "impl": "ours",
+            "value": round(c["flops"] * args.steps / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "chunked_prefill: 32 seqs, lengths U[1024,4096], last 512 tokens as queries, "
+                                   "block 16, 32 q / 8 KV heads, d128, bf16"},
+            "prefill_tokens_per_s": round(c["rows"] * args.steps / (ms * 1e-3), 1),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "traffic": None, "kernel": "paged_prefill_kernel",
+                         "kernel_ms": round(kern_ms, 4), "flops_per_launch": c["flops"],
+                         "peak_source": "measured" if "bf16_tflops" in peaks else "fallback"},
+            "gpu_launches": pa.pa_launch_count() - lc0, "clocks": clk, "device_error": pa.pa_device_error()}
+    if not args.no_cpu_baseline:
+        import oracle
+        import time as _t
+        from synthetic import values as sv
+        s0 = 0
+        L, C = c["lens_list"][s0], c["chunks"][s0]
+        k = sv.rows(sv.KIND_K, r["seed"], 0, np.zeros(L, np.int64), np.arange(L), sh.num_kv_heads, sh.head_dim,
+                    sh.kv_scale, sh.dtype)
+        v = sv.rows(sv.KIND_V, r["seed"], 0, np.zeros(L, np.int64), np.arange(L), sh.num_kv_heads, sh.head_dim,
+                    sh.kv_scale, sh.dtype)
+        nblk = -(-L // sh.block_size)
+        pad = nblk * sh.block_size - L
+        shp = (nblk, sh.block_size, sh.num_kv_heads, sh.head_dim)
+        kp = np.concatenate([k, np.zeros((pad,) + k.shape[1:], k.dtype)]).reshape(shp).transpose(0, 2, 1, 3)
+        vp = np.concatenate([v, np.zeros((pad,) + v.shape[1:], v.dtype)]).reshape(shp).transpose(0, 2, 1, 3)
+        qq = sv.rows(sv.KIND_Q, r["seed"], 0, np.zeros(C, np.int64), np.arange(L - C, L), sh.num_q_heads,
+                     sh.head_dim, sh.q_scale, sh.dtype)
+        fl = sum(4.0 * (L - C + i + 1) * sh.num_q_heads * sh.head_dim for i in range(C))
+        reps, dt = 0, 0.0
+        while reps == 0 or dt < args.cpu_seconds:
+            t = _t.perf_counter()
+            oracle.paged_prefill(np.ascontiguousarray(kp), np.ascontiguousarray(vp), sh.dtype,
+                                 np.arange(nblk, dtype=np.int32)[None], [L], [0, C], qq, scale)
+            dt += _t.perf_counter() - t
+            reps += 1
+        line["cpu_baseline"] = {"value": round(fl * reps / dt / 1e12, 6), "unit": "TFLOP/s",
+                                "cores": oracle.max_threads(), "kind": "oracle",
+                                "sample": f"fp64 oracle prefill of sequence 0 ({C} queries over {L} keys), "
+                                          f"repeated {reps}x for {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.workload == "swap":
         run_swap(args)
+        return
+    if args.workload == "prefill":
+        run_prefill(args)
         return
     if args.impl == "reference":
         run_reference(args)

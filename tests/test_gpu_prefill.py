@@ -120,3 +120,36 @@ def test_prefill_rejects_unsupported_shapes():
                                 torch.ones(1, dtype=torch.int32, device="cuda"),
                                 torch.tensor([0, 4], dtype=torch.int32, device="cuda"), 4, 0.1)
     assert e.value.status == pa.PA_ERR_UNSUPPORTED
+
+
+@pytest.mark.slow
+def test_chunked_prefill_workload_full_size_sampled():
+    """The benchmarked chunked-prefill workload (32 sequences, 512-token chunks) in the
+    launch configuration bench.py times; three sequences checked against the oracle on
+    regenerated histories."""
+    import bench
+    from synthetic import workloads as wl
+    r = wl.chunked_prefill()
+    sh = r["shape"]
+    c = bench.prefill_setup(torch, r)
+    out = torch.empty((c["rows"], sh.num_q_heads, sh.head_dim), dtype=torch.float32, device="cuda")
+    pa.pa_prefill_attention(c["cache"].pool, 0, c["q"], out, c["tables"], c["lens"], c["q_start"], c["max_q"],
+                            1 / math.sqrt(sh.head_dim))
+    got = out.cpu().numpy()
+    q_start = c["q_start"].cpu().numpy()
+    for s in (0, int(np.argmax(r["lens"])), len(r["lens"]) - 1):
+        L, C = int(r["lens"][s]), int(r["chunks"][s])
+        k = sv.rows(sv.KIND_K, r["seed"], 0, np.full(L, s), np.arange(L), sh.num_kv_heads, sh.head_dim,
+                    sh.kv_scale, sh.dtype)
+        v = sv.rows(sv.KIND_V, r["seed"], 0, np.full(L, s), np.arange(L), sh.num_kv_heads, sh.head_dim,
+                    sh.kv_scale, sh.dtype)
+        nblk = -(-L // 16)
+        pad = nblk * 16 - L
+        shp = (nblk, 16, sh.num_kv_heads, sh.head_dim)
+        kp = np.concatenate([k, np.zeros((pad,) + k.shape[1:], k.dtype)]).reshape(shp).transpose(0, 2, 1, 3)
+        vp = np.concatenate([v, np.zeros((pad,) + v.shape[1:], v.dtype)]).reshape(shp).transpose(0, 2, 1, 3)
+        q = sv.rows(sv.KIND_Q, r["seed"], 0, np.full(C, s), np.arange(L - C, L), sh.num_q_heads, sh.head_dim,
+                    sh.q_scale, sh.dtype)
+        ref = oracle.paged_prefill(np.ascontiguousarray(kp), np.ascontiguousarray(vp), sh.dtype,
+                                   np.arange(nblk, dtype=np.int32)[None], [L], [0, C], q, 1 / math.sqrt(sh.head_dim))
+        check_close(got[q_start[s]:q_start[s + 1]], ref, "f32", "bf16", f"chunked prefill seq {s}")
