@@ -1280,7 +1280,8 @@ pa_status pa_prefill_attention(pa_pool *pool, int32_t layer, const void *q, void
     if (group != 1 && group != 2 && group != 4 && group != 8)
         return fail(PA_ERR_UNSUPPORTED, "pa_prefill_attention: query heads per KV head must be 1, 2, 4 or 8");
     if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: scale must be finite");
-    const int64_t tiles = ((int64_t)max_q_len * group + prefill::kRows - 1) / prefill::kRows;
+    const int64_t tiles = ((int64_t)max_q_len * group + prefill::kTiles * prefill::kRows - 1) /
+                          (prefill::kTiles * prefill::kRows);
     if (tiles > INT32_MAX || c.num_kv_heads > 65535 || n_seqs > 65535)
         return fail(PA_ERR_UNSUPPORTED, "pa_prefill_attention: grid too large");
     pa_status st = ensure_tensor_maps(pool);

@@ -8,37 +8,42 @@
 // already in the paged cache; query i of the chunk (absolute position L - C + i)
 // attends to keys 0 .. L - C + i, read through the block table.
 //
-// One CTA per (128-row query tile, KV head, sequence).  Rows are (token, query head of
-// the GQA group) pairs, row = token * G + head, so every query head of the group
-// shares each key/value tile.  Per 64-key tile (64 / block_size blocks):
-//   TMA (2-D tensor loads, 128-byte swizzle) of K and V into a 2-stage ring;
-//   S = Q K^T        tcgen05.mma kind::f16, M=128, N=64, K=head_dim, D in TMEM;
-//   softmax          each thread owns one row = one TMEM lane: tcgen05.ld of its 64
-//                    scores, causal / length mask by select, base-2 online softmax
-//                    with a lazily moved maximum (rescales O in TMEM only when a score
-//                    passes the running maximum by 2^8), P split into a 16-bit high
-//                    part and the 16-bit rounding of the remainder, both written to
-//                    shared memory in the K-major swizzled layout;
-//   O += P V         tcgen05.mma kind::f16, M=128, N=head_dim, K=64, once with the
-//                    high part and once with the remainder (about 16 bits of each
-//                    weight survive), V read as an MN-major operand straight from the
-//                    TMA tile.
-// Key rows past the sequence end are zeroed in shared memory before P V (their weight
-// is 0, but 0 * NaN would not be).  Version 1 runs S, softmax and P V one after the
-// other; the TMA ring prefetches the next tile meanwhile.
+// One CTA per (256 query rows, KV head, sequence): two 128-row tiles A and B whose rows
+// are (token, query head of the GQA group) pairs, row = token * G + head, so every
+// query head of the group shares each key/value tile.  Warp roles:
+//   warps 0-3 / 4-7  softmax of tile A / B: thread = row = TMEM lane; tcgen05.ld of the
+//                    row's 64 scores, causal / length mask by select, base-2 online
+//                    softmax with a lazily moved maximum (the O row is rescaled in TMEM
+//                    only when a score passes the running maximum by 2^8), P split into
+//                    a 16-bit high part and the 16-bit rounding of the remainder, both
+//                    written to shared memory in the K-major 128-byte-swizzled layout;
+//   warp 8           tensor-core issue (one lane): S_t = Q_t K^T (M=128, N=64) and
+//                    O_t += P_t V (M=128, N=head_dim, hi and lo parts) in TMEM;
+//   warp 9           TMA producer: 64-key tiles of K and V (2-D tensor loads, 128-byte
+//                    swizzle) into a 2-stage ring, walking the block table.
+// The two tiles ping-pong: while one warpgroup computes exponentials the tensor core
+// works on the other tile.  Every hand-off is an mbarrier; every wait is bounded and
+// sets a shared abort flag that all roles check; TMEM is always freed.  Key rows past
+// the sequence end are zeroed in shared memory before P V (weight 0, but 0 * NaN would
+// not be 0).
 namespace prefill {
 
-constexpr int kRows = 128;           // MMA M: query rows of a tile
-constexpr int kKeys = 64;            // keys per tile
-constexpr int kThreads = 128;        // one thread per row / TMEM lane
+constexpr int kRows = 128;           // MMA M: rows of one query tile
+constexpr int kTiles = 2;            // query tiles per CTA (ping-pong)
+constexpr int kKeys = 64;            // keys per K/V tile
+constexpr int kSoftmaxThreads = kTiles * kRows;
+constexpr int kThreads = kSoftmaxThreads + 64;   // + tensor-core issue warp + TMA warp
+constexpr int kMmaWarp = kSoftmaxThreads / 32, kTmaWarp = kMmaWarp + 1;
 constexpr int kD = 128;              // head_dim
-constexpr uint32_t kTmemCols = 256;  // O in [0, 128), S in [128, 192)
-constexpr uint32_t kOCol = 0, kSCol = 128;
-constexpr int kQBytes = kRows * kD * 2;         // 32 KB: [2 halves][128 rows][128 B]
+constexpr uint32_t kTmemCols = 512;  // O_A [0,128) O_B [128,256) S_A [256,320) S_B [320,384)
+constexpr uint32_t kOCol = 0, kSCol = 256;
+constexpr int kQBytes = kRows * kD * 2;         // 32 KB per tile: [2 halves][128 rows][128 B]
 constexpr int kKVBytes = kKeys * kD * 2;        // 16 KB: [2 halves][64 rows][128 B]
-constexpr int kPBytes = kRows * kKeys * 2;      // 16 KB: [128 rows][128 B], high and low parts
+constexpr int kPBytes = kRows * kKeys * 2;      // 16 KB per part: [128 rows][128 B]
 constexpr int kStages = 2;
-constexpr int kSmemBytes = 1024 + kQBytes + kStages * 2 * kKVBytes + 2 * kPBytes + 64;
+constexpr int kNumBars = 3 * kTiles + 2 * kStages;
+constexpr int kSmemBytes = 1024 + kTiles * kQBytes + kStages * 2 * kKVBytes + kTiles * 2 * kPBytes +
+                           kNumBars * 8 + 16;
 
 // --- tcgen05 wrappers --------------------------------------------------------------
 // Shared-memory matrix descriptor, 128-byte swizzle: start address, leading and stride
@@ -112,21 +117,23 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Bounded wait polled by every thread; a thread that gives up sets the abort flag so
-// the others stop polling.  Callers combine the results with __syncthreads_and, so
-// the whole CTA takes the same branch.
-__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
-            raise_error(kErrTimeout);
-            *abort_flag = 1;
+// Bounded wait for a whole warp (lanes leave together); gives up when another role has
+// set the abort flag or after kWaitLimitNs, setting the flag itself then.
+__device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        const bool done = mbar_try_wait(bar, parity);
+        if (__all_sync(0xffffffffu, done)) return true;
+        if (it == 0) t0 = global_timer_ns();
+        const bool give_up = *abort_flag || global_timer_ns() - t0 > kWaitLimitNs;
+        if (__any_sync(0xffffffffu, give_up)) {
+            if ((threadIdx.x & 31) == 0 && !*abort_flag) {
+                raise_error(kErrTimeout);
+                *abort_flag = 1;
+            }
             return false;
         }
     }
-    return true;
 }
 
 template <typename T>
@@ -159,240 +166,287 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
     constexpr uint32_t IDESC_O = instr_desc(Fmt<T>::code, kRows, kD, 0, 1);
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
-    unsigned char *sQ = smem;
-    unsigned char *sK = sQ + kQBytes;                    // stage st: sK + st * 2 * kKVBytes
-    unsigned char *sP = sK + kStages * 2 * kKVBytes;          // high part; low part follows
-    uint64_t *full = reinterpret_cast<uint64_t *>(sP + 2 * kPBytes);   // [kStages]
-    uint64_t *mma_bar = full + kStages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 1);
+    unsigned char *sQ = smem;                                       // tile t at t * kQBytes
+    unsigned char *sKV = sQ + kTiles * kQBytes;                     // stage st: K then V
+    unsigned char *sP = sKV + kStages * 2 * kKVBytes;               // tile t: hi, lo
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sP + kTiles * 2 * kPBytes);
+    uint64_t *kv_full = bars, *kv_empty = bars + kStages;
+    uint64_t *s_full = bars + 2 * kStages, *p_full = s_full + kTiles, *o_done = p_full + kTiles;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int s = blockIdx.z;
     const int g = blockIdx.y;
-    const int qt = blockIdx.x;
     const int group = p.num_q_heads / p.num_kv_heads;
-    const int tokens_per_tile = kRows / group;
+    const int tokens_per_cta = kTiles * kRows / group;
     const int q0 = p.q_start[s];
     const int C = p.q_start[s + 1] - q0;
-    const int t0 = qt * tokens_per_tile;
+    const int t0 = blockIdx.x * tokens_per_cta;
     if (t0 >= C) return;
-    int L = p.lens[s];
+    const int L = p.lens[s];
     const int nblk = (L + B - 1) / B;
     if (L < 1 || C > L || nblk > p.max_blocks) {
         if (threadIdx.x == 0) raise_error(kErrBadLen);
         return;
     }
-    const int P0 = L - C;                                  // position of the chunk's first token
-    const int t_last = min(C, t0 + tokens_per_tile) - 1;
-    const int n_tiles = (P0 + t_last) / kKeys + 1;         // keys 0 .. P0 + t_last
+    const int P0 = L - C;                                    // position of the chunk's first token
+    const int t_last = min(C, t0 + tokens_per_cta) - 1;
+    const int n_tiles = (P0 + t_last) / kKeys + 1;           // keys 0 .. P0 + t_last
+    const bool has_b = t0 + kRows / group < C;               // tile B holds at least one token
+    const int n_qt = has_b ? 2 : 1;
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
-    const int32_t *trow = p.tables + (size_t)s * p.max_blocks;
+    const int lane = tid & 31;
 
     if (tid == 0) {
-        for (int i = 0; i < kStages; ++i) mbar_init(&full[i], 1);
-        mbar_init(mma_bar, 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
+        }
+        for (int t = 0; t < kTiles; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&p_full[t], 4);        // the four warps of the tile's softmax group
+            mbar_init(&o_done[t], 1);
+        }
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (warp == 0) {   // TMEM: one warp allocates (and later frees) for the CTA
+    if (warp == kMmaWarp) {   // TMEM: the issuing warp allocates and frees
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
                      "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-
-    // K/V tile loads (thread 0): blocks past the sequence end load the first block
-    // instead (finite data; masked and zeroed before use).
-    auto issue_tile = [&](int j) {
-        const int st = j % kStages;
-        unsigned char *k_dst = sK + st * 2 * kKVBytes;
-        unsigned char *v_dst = k_dst + kKVBytes;
-        mbar_arrive_expect_tx(&full[st], 2 * kKVBytes);
-        for (int b = 0; b < BLOCKS_PER_TILE; ++b) {
-            const int lb = j * BLOCKS_PER_TILE + b;
-            int blk = trow[lb < nblk ? lb : 0];
-            if ((unsigned)blk >= (unsigned)p.num_blocks) {
-                raise_error(kErrBadBlock);
-                blk = 0;
-            }
-            const int row = ((p.layer * p.num_blocks + blk) * p.num_kv_heads + g) * B;
-            for (int h = 0; h < 2; ++h) {
-                tma_load_2d(k_dst + h * (kKVBytes / 2) + b * B * 128, &p.tmap_k, h * 64, row, &full[st]);
-                tma_load_2d(v_dst + h * (kKVBytes / 2) + b * B * 128, &p.tmap_v, h * 64, row, &full[st]);
-            }
-        }
-    };
-
-    // Q tile: row r = token * G + head; rows past the chunk are zero
-    const int my_t = t0 + tid / group;
-    const int my_h = g * group + tid % group;
-    const bool row_valid = my_t < C;
-    {
+    // query rows: tile t = tid / 128, row r = tid % 128; rows past the chunk are zero
+    const int qtile = tid / kRows;
+    const int row = tid % kRows;
+    const int my_t = t0 + (qtile * kRows + row) / group;
+    const int my_h = g * group + row % group;
+    const bool row_valid = tid < kSoftmaxThreads && my_t < C;
+    if (tid < kSoftmaxThreads) {
         const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.q) +
                                                             ((size_t)(q0 + (row_valid ? my_t : 0)) * p.num_q_heads + my_h) * kD);
+        unsigned char *dst = sQ + qtile * kQBytes;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
             const uint4 v = row_valid ? src[c] : make_uint4(0, 0, 0, 0);
             const int half = c >> 3, cc = c & 7;
-            *reinterpret_cast<uint4 *>(sQ + half * (kQBytes / 2) + tid * 128 + ((cc ^ (tid & 7)) << 4)) = v;
+            *reinterpret_cast<uint4 *>(dst + half * (kQBytes / 2) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
         }
+        fence_proxy_async();
     }
-    fence_proxy_async();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    if (tid == 0) {
-        issue_tile(0);
-        if (n_tiles > 1) issue_tile(1);
-    }
 
-    const int kmax = row_valid ? P0 + my_t : -1;            // last key this row may see
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const float sl = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
-    const uint32_t qaddr = smem_addr(sQ), paddr = smem_addr(sP);
-    bool ok = true;
-
-    for (int j = 0; j < n_tiles && ok; ++j) {
-        const int st = j % kStages;
-        unsigned char *k_st = sK + st * 2 * kKVBytes;
-        unsigned char *v_st = k_st + kKVBytes;
-        ok = __syncthreads_and(wait_all(&full[st], (j / kStages) & 1, abort_flag));
-        if (!ok) break;
-        // keys past the sequence end: zero their V rows (whole 128-byte rows, both halves)
-        const int first_bad = L - j * kKeys;
-        if (first_bad < kKeys) {
-            const int row = tid >> 1, half = tid & 1;
-            if (row >= first_bad) {
-                uint4 *dst = reinterpret_cast<uint4 *>(v_st + half * (kKVBytes / 2) + row * 128);
+    if (warp == kTmaWarp) {
+        // ---------------- producer: walk the table, keep the ring full
+        const int32_t *trow = p.tables + (size_t)s * p.max_blocks;
+        for (int j = 0; j < n_tiles; ++j) {
+            const int st = j % kStages;
+            if (j >= kStages && !wait_warp(&kv_empty[st], ((j / kStages) - 1) & 1, abort_flag)) break;
+            int blk = 0;
+            if (lane < BLOCKS_PER_TILE) {
+                const int lb = j * BLOCKS_PER_TILE + lane;
+                blk = trow[lb < nblk ? lb : 0];      // past the end: finite data, masked and zeroed
+                if ((unsigned)blk >= (unsigned)p.num_blocks) {
+                    raise_error(kErrBadBlock);
+                    blk = 0;
+                }
+            }
+            if (lane == 0) mbar_arrive_expect_tx(&kv_full[st], 2 * kKVBytes);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+            for (int b = 0; b < BLOCKS_PER_TILE; ++b) {
+                const int bb = __shfl_sync(0xffffffffu, blk, b);
+                if (lane == 0) {
+                    const int r0 = ((p.layer * p.num_blocks + bb) * p.num_kv_heads + g) * B;
+                    unsigned char *k_dst = sKV + st * 2 * kKVBytes;
+                    for (int h = 0; h < 2; ++h) {
+                        tma_load_2d(k_dst + h * (kKVBytes / 2) + b * B * 128, &p.tmap_k, h * 64, r0, &kv_full[st]);
+                        tma_load_2d(k_dst + kKVBytes + h * (kKVBytes / 2) + b * B * 128, &p.tmap_v, h * 64, r0,
+                                    &kv_full[st]);
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    } else if (warp == kMmaWarp) {
+        // ---------------- tensor-core issue
+        // wait for tile j's keys/values; zero value rows past the sequence end
+        auto ready = [&](int j) -> bool {
+            const int st = j % kStages;
+            if (!wait_warp(&kv_full[st], (j / kStages) & 1, abort_flag)) return false;
+            const int first_bad = L - j * kKeys;
+            if (first_bad < kKeys) {
+                unsigned char *v_st = sKV + st * 2 * kKVBytes + kKVBytes;
+                for (int rr = lane; rr < 2 * kKeys; rr += 32) {
+                    const int r = rr >> 1, half = rr & 1;
+                    if (r >= first_bad) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(v_st + half * (kKVBytes / 2) + r * 128);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                fence_proxy_async();
+                __syncwarp();
+            }
+            fence_after_sync();
+            return true;
+        };
+        auto issue_s = [&](int t, int j) {
+            if (lane == 0) {
+                const uint32_t qaddr = smem_addr(sQ + t * kQBytes);
+                const uint32_t kaddr = smem_addr(sKV + (j % kStages) * 2 * kKVBytes);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t a = smem_desc(qaddr + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
+                    const uint64_t b = smem_desc(kaddr + (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32, 16, 1024);
+                    umma(tmem + kSCol + t * kKeys, a, b, IDESC_S, kk > 0);
+                }
+                umma_commit(&s_full[t]);
+            }
+            __syncwarp();
+        };
+        auto issue_pv = [&](int t, int j) {
+            if (lane == 0) {
+                const uint32_t paddr = smem_addr(sP + t * 2 * kPBytes);
+                const uint32_t vaddr = smem_addr(sKV + (j % kStages) * 2 * kKVBytes + kKVBytes);
+#pragma unroll
+                for (int kk = 0; kk < kKeys / 16; ++kk) {
+                    const uint64_t b = smem_desc(vaddr + kk * 16 * 128, kKVBytes / 2, 1024);
+                    umma(tmem + kOCol + t * kD, smem_desc(paddr + kk * 32, 16, 1024), b, IDESC_O,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+                    umma(tmem + kOCol + t * kD, smem_desc(paddr + kPBytes + kk * 32, 16, 1024), b, IDESC_O, 1u);
+                }
+                umma_commit(&o_done[t]);
+            }
+            __syncwarp();
+        };
+        bool ok = ready(0);
+        if (ok)
+            for (int t = 0; t < n_qt; ++t) issue_s(t, 0);
+        for (int j = 0; j < n_tiles && ok; ++j) {
+            for (int t = 0; t < n_qt && ok; ++t) {
+                ok = wait_warp(&p_full[t], j & 1, abort_flag);   // softmax t read S_t(j), wrote P_t(j)
+                if (!ok) break;
+                fence_after_sync();
+                issue_pv(t, j);
+                if (j + 1 < n_tiles) {
+                    if (t == 0) ok = ready(j + 1);
+                    if (ok) issue_s(t, j + 1);
+                }
+            }
+            if (ok && lane == 0) umma_commit(&kv_empty[j % kStages]);
+            __syncwarp();
+        }
+    } else {
+        // ---------------- softmax of tile qtile, row = TMEM lane
+        const bool tile_used = qtile < n_qt;
+        const int kmax = row_valid ? P0 + my_t : -1;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t s_col = kSCol + qtile * kKeys, o_col = kOCol + qtile * kD;
+        unsigned char *p_hi = sP + qtile * 2 * kPBytes;
+        const float sl = p.scale_log2;
+        float m = -INFINITY, l = 0.f;
+        bool ok = tile_used;
+        for (int j = 0; j < n_tiles && ok; ++j) {
+            ok = wait_warp(&s_full[qtile], j & 1, abort_flag);
+            if (!ok) break;
+            fence_after_sync();
+            uint32_t sv[64];
+            {
+                uint32_t a[32], b[32];
+                tmem_ld32(tmem + lane_base + s_col, a);
+                tmem_ld32(tmem + lane_base + s_col + 32, b);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    sv[c] = a[c];
+                    sv[32 + c] = b[c];
+                }
+            }
+            const int key0 = j * kKeys;
+            float tmax = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                const float x = (key0 + c <= kmax && key0 + c < L) ? __uint_as_float(sv[c]) * sl : -INFINITY;
+                sv[c] = __float_as_uint(x);
+                tmax = fmaxf(tmax, x);
+            }
+            if (j > 0) {   // P_t(j-1) consumed and O_t settled before P_t and O_t are touched
+                ok = wait_warp(&o_done[qtile], (j - 1) & 1, abort_flag);
+                if (!ok) break;
+                fence_after_sync();
+            }
+            if (tmax > m + kRescaleThreshold) {
+                const float f = ex2(m - tmax);
+                if (j > 0) {
+#pragma unroll
+                    for (int c0 = 0; c0 < kD; c0 += 32) {
+                        uint32_t o[32];
+                        tmem_ld32(tmem + lane_base + o_col + c0, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+                        tmem_st32(tmem + lane_base + o_col + c0, o);
+                    }
+                    tmem_wait_st();
+                }
+                l *= f;
+                m = tmax;
+            }
+            const bool any = m != -INFINITY;
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+                uint32_t w[4], r[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = __uint_as_float(sv[c8 * 8 + 2 * e]);
+                    const float x1 = __uint_as_float(sv[c8 * 8 + 2 * e + 1]);
+                    const float p0 = any ? ex2(x0 - m) : 0.f;
+                    const float p1 = any ? ex2(x1 - m) : 0.f;
+                    w[e] = Mma<T>::pack(p0, p1);
+                    r[e] = Mma<T>::pack(p0 - Mma<T>::low(w[e]), p1 - Mma<T>::high(w[e]));
+                    l += p0 + p1;
+                }
+                const int off = row * 128 + ((c8 ^ (row & 7)) << 4);
+                *reinterpret_cast<uint4 *>(p_hi + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(p_hi + kPBytes + off) = make_uint4(r[0], r[1], r[2], r[3]);
             }
             fence_proxy_async();
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[qtile]);
         }
-        fence_before_sync();
-        __syncthreads();
-        // S = Q K^T
-        if (tid == 0) {
+        if (ok) ok = wait_warp(&o_done[qtile], (n_tiles - 1) & 1, abort_flag);
+        if (ok) {
             fence_after_sync();
-            const uint32_t kaddr = smem_addr(k_st);
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const size_t orow = ((size_t)(q0 + my_t) * p.num_q_heads + my_h) * kD;
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-                const uint64_t a = smem_desc(qaddr + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
-                const uint64_t b = smem_desc(kaddr + (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32, 16, 1024);
-                umma(tmem + kSCol, a, b, IDESC_S, kk > 0);
-            }
-            umma_commit(mma_bar);
-        }
-        ok = __syncthreads_and(wait_all(mma_bar, 0, abort_flag));
-        if (!ok) break;
-        fence_after_sync();
-        uint32_t sv[64];
-        {
-            uint32_t a[32], b[32];
-            tmem_ld32(tmem + lane_base + kSCol, a);
-            tmem_ld32(tmem + lane_base + kSCol + 32, b);
-            tmem_wait_ld();
+            for (int c0 = 0; c0 < kD; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_base + o_col + c0, o);
+                tmem_wait_ld();
+                if (row_valid) {
+                    if (p.out_f32) {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + orow + c0);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                sv[c] = a[c];
-                sv[32 + c] = b[c];
-            }
-        }
-        // mask, scale, running maximum
-        const int key0 = j * kKeys;
-        float tmax = -INFINITY;
+                        for (int c = 0; c < 32; c += 4)
+                            dst[c / 4] = make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
+                                                     __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+                    } else {
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<T *>(p.out) + orow + c0);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-            const float x = (key0 + c <= kmax && key0 + c < L) ? __uint_as_float(sv[c]) * sl : -INFINITY;
-            sv[c] = __float_as_uint(x);
-            tmax = fmaxf(tmax, x);
-        }
-        if (tmax > m + kRescaleThreshold) {
-            const float f = ex2(m - tmax);     // 0 while nothing has been accumulated
-            if (j > 0) {                       // O holds earlier tiles: scale this row in TMEM
+                        for (int c = 0; c < 32; c += 8) {
+                            uint32_t w[4];
 #pragma unroll
-                for (int c0 = 0; c0 < kD; c0 += 32) {
-                    uint32_t o[32];
-                    tmem_ld32(tmem + lane_base + kOCol + c0, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
-                    tmem_st32(tmem + lane_base + kOCol + c0, o);
-                }
-                tmem_wait_st();
-            }
-            l *= f;
-            m = tmax;
-        }
-        // P as high + low 16-bit parts (K-major swizzled) and the row sum
-        const bool any = m != -INFINITY;
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-            uint32_t w[4], r[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float x0 = __uint_as_float(sv[c8 * 8 + 2 * e]);
-                const float x1 = __uint_as_float(sv[c8 * 8 + 2 * e + 1]);
-                const float p0 = any ? ex2(x0 - m) : 0.f;
-                const float p1 = any ? ex2(x1 - m) : 0.f;
-                w[e] = Mma<T>::pack(p0, p1);
-                r[e] = Mma<T>::pack(p0 - Mma<T>::low(w[e]), p1 - Mma<T>::high(w[e]));
-                l += p0 + p1;
-            }
-            const int off = tid * 128 + ((c8 ^ (tid & 7)) << 4);
-            *reinterpret_cast<uint4 *>(sP + off) = make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4 *>(sP + kPBytes + off) = make_uint4(r[0], r[1], r[2], r[3]);
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-        // O += P V
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t vaddr = smem_addr(v_st);
-#pragma unroll
-            for (int kk = 0; kk < kKeys / 16; ++kk) {
-                const uint64_t b = smem_desc(vaddr + kk * 16 * 128, kKVBytes / 2, 1024);
-                umma(tmem + kOCol, smem_desc(paddr + kk * 32, 16, 1024), b, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
-                umma(tmem + kOCol, smem_desc(paddr + kPBytes + kk * 32, 16, 1024), b, IDESC_O, 1u);
-            }
-            umma_commit(mma_bar);
-        }
-        ok = __syncthreads_and(wait_all(mma_bar, 1, abort_flag));
-        if (!ok) break;
-        fence_after_sync();
-        if (tid == 0 && j + kStages < n_tiles) issue_tile(j + kStages);
-    }
-
-    if (ok) {
-        // O / l for this row
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        const size_t orow = ((size_t)(q0 + my_t) * p.num_q_heads + my_h) * kD;
-#pragma unroll
-        for (int c0 = 0; c0 < kD; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_base + kOCol + c0, o);
-            tmem_wait_ld();
-            if (row_valid) {
-                if (p.out_f32) {
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + orow + c0);
-#pragma unroll
-                    for (int c = 0; c < 32; c += 4)
-                        dst[c / 4] = make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
-                                                 __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
-                } else {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<T *>(p.out) + orow + c0);
-#pragma unroll
-                    for (int c = 0; c < 32; c += 8) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            w[e] = Mma<T>::pack(__uint_as_float(o[c + 2 * e]) * inv,
-                                                __uint_as_float(o[c + 2 * e + 1]) * inv);
-                        dst[c / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+                            for (int e = 0; e < 4; ++e)
+                                w[e] = Mma<T>::pack(__uint_as_float(o[c + 2 * e]) * inv,
+                                                    __uint_as_float(o[c + 2 * e + 1]) * inv);
+                            dst[c / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
                     }
                 }
             }
@@ -400,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
     }
     fence_before_sync();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kMmaWarp) {
         fence_after_sync();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                      : "memory");
