@@ -367,13 +367,18 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                 }
             }
             const int key0 = j * kKeys;
-            float tmax = -INFINITY;
+            // interior tiles need no mask; the last ones mask by select (keys past this
+            // row's position or past the sequence end get weight 0)
+            const bool full_tile = key0 + kKeys - 1 <= kmax && key0 + kKeys <= L;
+            if (!full_tile) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const float x = (key0 + c <= kmax && key0 + c < L) ? __uint_as_float(sv[c]) * sl : -INFINITY;
-                sv[c] = __float_as_uint(x);
-                tmax = fmaxf(tmax, x);
+                for (int c = 0; c < 64; ++c)
+                    if (!(key0 + c <= kmax && key0 + c < L)) sv[c] = __float_as_uint(-INFINITY);
             }
+            float smax = -INFINITY;                 // on raw scores: scale > 0 keeps the order
+#pragma unroll
+            for (int c = 0; c < 64; ++c) smax = fmaxf(smax, __uint_as_float(sv[c]));
+            const float tmax = smax * sl;
             if (j > 0) {   // P_t(j-1) consumed and O_t settled before P_t and O_t are touched
                 ok = wait_warp(&o_done[qtile], (j - 1) & 1, abort_flag);
                 if (!ok) break;
@@ -396,24 +401,25 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                 l *= f;
                 m = tmax;
             }
-            const bool any = m != -INFINITY;
+            // p = 2^(s * scale_log2 - m): one FMA and one ex2 per score (-inf -> 0)
+            const float neg_m = m == -INFINITY ? 0.f : -m;
+            float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8) {
                 uint32_t w[4], r[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float x0 = __uint_as_float(sv[c8 * 8 + 2 * e]);
-                    const float x1 = __uint_as_float(sv[c8 * 8 + 2 * e + 1]);
-                    const float p0 = any ? ex2(x0 - m) : 0.f;
-                    const float p1 = any ? ex2(x1 - m) : 0.f;
+                    const float p0 = ex2(fmaf(__uint_as_float(sv[c8 * 8 + 2 * e]), sl, neg_m));
+                    const float p1 = ex2(fmaf(__uint_as_float(sv[c8 * 8 + 2 * e + 1]), sl, neg_m));
                     w[e] = Mma<T>::pack(p0, p1);
                     r[e] = Mma<T>::pack(p0 - Mma<T>::low(w[e]), p1 - Mma<T>::high(w[e]));
-                    l += p0 + p1;
+                    lp[e] += p0 + p1;
                 }
                 const int off = row * 128 + ((c8 ^ (row & 7)) << 4);
                 *reinterpret_cast<uint4 *>(p_hi + off) = make_uint4(w[0], w[1], w[2], w[3]);
                 *reinterpret_cast<uint4 *>(p_hi + kPBytes + off) = make_uint4(r[0], r[1], r[2], r[3]);
             }
+            l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
             fence_proxy_async();
             fence_before_sync();
             __syncwarp();
