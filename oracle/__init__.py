@@ -9,8 +9,12 @@ bench.py's CPU-baseline leg may import it.
                                attention in double precision (oracle.c).
 * ``block_manager``         -- free stack, refcounts, tables, copy-on-write (Python).
 * ``cache_model``           -- where appended rows and copied blocks land (numpy).
+* ``fp8``                   -- E4M3 codes with per-row power-of-two scales: encode,
+                               decode, row quantisation (numpy).
+* ``paged_decode_fp8``      -- decode attention over an FP8 cache: dequantise exactly,
+                               then the same fp64 attention.
 
-Parity status of each function is recorded with its tests: all three are pinned
+Parity status of each function is recorded with its tests: all are pinned
 (closed forms and page figures, exhaustive decoder checks, brute force, a library
 routine, planted-mistake checks).
 """
@@ -20,10 +24,10 @@ import ctypes
 
 import numpy as np
 
-from . import block_manager, cache_model  # noqa: F401
+from . import block_manager, cache_model, fp8  # noqa: F401
 from .build import build as _build
 
-_CODES = {"f32": 0, "f16": 1, "bf16": 2}
+_CODES = {"f32": 0, "f16": 1, "bf16": 2, "f64": 3}
 _lib = None
 
 
@@ -111,6 +115,21 @@ def paged_prefill(k_layer: np.ndarray, v_layer: np.ndarray, dtype: str, tables, 
     if rc != 0:
         raise ValueError("oracle_paged_prefill rejected its arguments")
     return out
+
+
+def paged_decode_fp8(k_codes: np.ndarray, v_codes: np.ndarray, k_scales: np.ndarray, v_scales: np.ndarray,
+                     tables, lens, q: np.ndarray, q_dtype: str, scale: float, n_threads: int = 0) -> np.ndarray:
+    """fp64 paged decode attention over an FP8 cache (one layer).
+
+    k_codes, v_codes: [num_blocks][num_kv_heads][block_size][head_dim] E4M3 codes;
+    k_scales, v_scales: [num_blocks][num_kv_heads][block_size] scale bytes; q in its
+    own storage type ``q_dtype``.  Every cached value is dequantised exactly
+    (fp8.dequantize), then attention runs as in ``paged_decode``.
+    """
+    k = np.ascontiguousarray(fp8.dequantize(k_codes, k_scales))
+    v = np.ascontiguousarray(fp8.dequantize(v_codes, v_scales))
+    q64 = np.ascontiguousarray(widen(q, q_dtype))
+    return paged_decode(k, v, "f64", tables, lens, q64, scale, n_threads)
 
 
 def max_threads() -> int:

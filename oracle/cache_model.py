@@ -14,6 +14,12 @@ way the pages describe:
   copied, and copying the whole block keeps every earlier slot valid).
 
 Writes are bit copies, so the GPU pools must match these arrays exactly.
+
+FP8 pools (``dtype == "fp8"``) hold E4M3 codes and, beside them, one scale byte per
+(token, KV head) row in arrays [num_layers][num_blocks][num_kv_heads][block_size];
+an appended row is quantised by ``oracle.fp8.quantize_rows`` (the format and the
+scale rule are stated there), and block copies and swaps carry the scales with the
+codes.
 """
 from __future__ import annotations
 
@@ -21,13 +27,41 @@ import numpy as np
 
 from synthetic.values import ELEM_BYTES
 
+from .fp8 import quantize_rows
+
 _NP = {"f32": np.float32, "f16": np.float16, "bf16": np.uint16}
 
 
 def empty_pools(num_layers, num_blocks, num_kv_heads, block_size, head_dim, dtype):
     shape = (num_layers, num_blocks, num_kv_heads, block_size, head_dim)
+    if dtype == "fp8":
+        return np.zeros(shape, np.uint8), np.zeros(shape, np.uint8)
     assert ELEM_BYTES[dtype] == np.dtype(_NP[dtype]).itemsize
     return np.zeros(shape, _NP[dtype]), np.zeros(shape, _NP[dtype])
+
+
+def empty_scales(num_layers, num_blocks, num_kv_heads, block_size):
+    """Scale-byte arrays of an FP8 pool (K and V), [layers][blocks][kv heads][block_size]."""
+    shape = (num_layers, num_blocks, num_kv_heads, block_size)
+    return np.zeros(shape, np.uint8), np.zeros(shape, np.uint8)
+
+
+def append_rows_fp8(k_pool, v_pool, k_scales, v_scales, layer, slots, k_rows, v_rows, act_dtype):
+    """Quantise row i of k_rows / v_rows ([n][Hkv][d], storage of ``act_dtype``) and
+    write its codes and scale bytes into slot slots[i] of ``layer``."""
+    from . import widen                      # the oracle's own exact decoders
+    kc, ks = quantize_rows(widen(k_rows, act_dtype).astype(np.float32))
+    vc, vs = quantize_rows(widen(v_rows, act_dtype).astype(np.float32))
+    block_size = k_pool.shape[3]
+    for i, slot in enumerate(slots):
+        slot = int(slot)
+        if slot < 0:
+            continue
+        blk, off = divmod(slot, block_size)
+        k_pool[layer, blk, :, off, :] = kc[i]
+        v_pool[layer, blk, :, off, :] = vc[i]
+        k_scales[layer, blk, :, off] = ks[i]
+        v_scales[layer, blk, :, off] = vs[i]
 
 
 def append_rows(k_pool, v_pool, layer, slots, k_rows, v_rows):
@@ -47,6 +81,37 @@ def copy_blocks(k_pool, v_pool, pairs):
     for src, dst in pairs:
         k_pool[:, int(dst)] = k_pool[:, int(src)]
         v_pool[:, int(dst)] = v_pool[:, int(src)]
+
+
+def copy_scales(k_scales, v_scales, pairs):
+    """The scale bytes travel with a copied FP8 block, every layer."""
+    for src, dst in pairs:
+        k_scales[:, int(dst)] = k_scales[:, int(src)]
+        v_scales[:, int(dst)] = v_scales[:, int(src)]
+
+
+def swap_buffer_fp8(k_pool, v_pool, k_scales, v_scales, blocks):
+    """Host copy of a swapped-out sequence of an FP8 pool, as bytes: for block i in
+    logical order and each layer, the K codes [heads][block_size][dim], the V codes,
+    then the K scale bytes [heads][block_size] and the V scale bytes (reading: the
+    scales ride in the same block-major record as their codes)."""
+    out = []
+    for b in blocks:
+        for layer in range(k_pool.shape[0]):
+            out += [k_pool[layer, int(b)].ravel(), v_pool[layer, int(b)].ravel(),
+                    k_scales[layer, int(b)].ravel(), v_scales[layer, int(b)].ravel()]
+    return np.concatenate(out) if out else np.zeros(0, np.uint8)
+
+
+def swap_restore_fp8(k_pool, v_pool, k_scales, v_scales, blocks, buf):
+    nl, _, h, bs, d = k_pool.shape
+    pos = 0
+    for b in blocks:
+        for layer in range(nl):
+            for arr, n, shape in ((k_pool, h * bs * d, (h, bs, d)), (v_pool, h * bs * d, (h, bs, d)),
+                                  (k_scales, h * bs, (h, bs)), (v_scales, h * bs, (h, bs))):
+                arr[layer, int(b)] = buf[pos:pos + n].reshape(shape)
+                pos += n
 
 
 def swap_buffer(k_pool, v_pool, blocks):

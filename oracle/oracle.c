@@ -19,7 +19,8 @@
  *   z_j    = scale * sum_i q[s][h][i] * K_s[j][i]
  *   o[i]   = sum_j exp(z_j - max z) V_s[j][i] / sum_j exp(z_j - max z)
  * all in double precision, after widening the stored fp32/fp16/bf16 values
- * exactly to double.
+ * exactly to double (or taking already-decoded double values as they are, which is
+ * how the FP8 cache's dequantised values come in).
  *
  * Pool layout of one layer: [num_blocks][num_kv_heads][block_size][head_dim].
  * Reading taken where the pages are silent: softmax scale is a parameter
@@ -33,7 +34,7 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_F32 = 0, ORACLE_F16 = 1, ORACLE_BF16 = 2 };
+enum { ORACLE_F32 = 0, ORACLE_F16 = 1, ORACLE_BF16 = 2, ORACLE_F64 = 3 };
 
 /* IEEE 754 binary16 -> double, from the format's definition:
  * 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
@@ -66,6 +67,7 @@ static double load_elem(const void *base, int dtype, size_t idx)
     switch (dtype) {
     case ORACLE_F32: return (double)((const float *)base)[idx];
     case ORACLE_F16: return oracle_half_to_double(((const uint16_t *)base)[idx]);
+    case ORACLE_F64: return ((const double *)base)[idx];   /* already-decoded values */
     default:         return oracle_bf16_to_double(((const uint16_t *)base)[idx]);
     }
 }
