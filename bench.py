@@ -57,6 +57,9 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seqs", type=int, default=24)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for the CPU baseline")
+    ap.add_argument("--kv-dtype", default="native", choices=["native", "fp8"],
+                    help="native: the workload's 16-bit cache; fp8: E4M3 codes + per-row scale bytes "
+                         "(queries and appended rows keep the workload's type)")
     ap.add_argument("--prefix-cache", default="on", choices=["on", "off"],
                     help="shared_prompt workload: share the cached system-prompt blocks at admission")
     a = ap.parse_args(argv)
@@ -64,6 +67,9 @@ def parse(argv=None):
         a.steps = 8 if a.workload.startswith("large_pool") or a.workload in ("swap", "prefill") else 64
     if a.split is None:
         a.split = DEFAULT_SPLIT[a.workload]
+    if a.kv_dtype == "fp8" and a.workload not in ("continuous_batch", "large_pool_b16", "large_pool_b32",
+                                                    "worked_example"):
+        ap.error("--kv-dtype fp8 runs the continuous_batch, large_pool and worked_example workloads")
     return a
 
 
@@ -221,7 +227,8 @@ class Replica:
     """One GPU's decode state: pools, block manager, sequences, and every step's inputs
     generated in HBM before timing starts."""
 
-    def __init__(self, torch, workload, recipe, total_steps, split, device, e2e_from, prefix_cache=True):
+    def __init__(self, torch, workload, recipe, total_steps, split, device, e2e_from, prefix_cache=True,
+                 kv_fp8=False):
         from paged_kv_cache_403_b200.engine import PagedCache
         from paged_kv_cache_403_b200.runners import DeviceGen, prefill
         import paged_kv_cache_403_b200 as pa
@@ -230,7 +237,12 @@ class Replica:
         sh = self.shape
         self.NL = sh.num_layers
         self.split, self.device = split, device
-        self.cache = PagedCache.from_shape(sh, recipe["order"], device)
+        self.kv_fp8 = kv_fp8
+        if kv_fp8:
+            self.cache = PagedCache(sh.num_layers, sh.num_blocks, sh.block_size, sh.num_kv_heads, sh.head_dim,
+                                    "fp8", recipe["order"], device, act_dtype=sh.dtype)
+        else:
+            self.cache = PagedCache.from_shape(sh, recipe["order"], device)
         gen = DeviceGen(recipe["seed"], sh, device)
         self.prompt_start = lambda plen: 0          # first prompt position an admission appends
         self.system_keys = None
@@ -426,8 +438,9 @@ class Replica:
             self.cache.free(self.sids[slot])
         # accounting: bytes decode attention reads / writes this step (all layers)
         L = lens.numpy().astype(np.int64)
-        e = 2
-        kv = self.NL * int((2 * L * sh.num_kv_heads * sh.head_dim * e).sum())
+        e = 2                                                  # bytes of a query / output element
+        row = sh.head_dim + 1 if self.kv_fp8 else sh.head_dim * e   # cached bytes of one (token, head) row
+        kv = self.NL * int((2 * L * sh.num_kv_heads * row).sum())
         alg = kv + self.NL * (2 * n * sh.num_q_heads * sh.head_dim * e + int((4 * -(-L // sh.block_size)).sum())
                               + 4 * n)
         self.kv_bytes.append(kv)
@@ -463,7 +476,7 @@ def run_ours(args):
     total = W + K + (K if e2e else 0)
     recipe = make_recipe(args.workload, replica_seed(rank), total)
     rep = Replica(torch, args.workload, recipe, total, args.split, device, W + K if e2e else None,
-                  prefix_cache=args.prefix_cache == "on")
+                  prefix_cache=args.prefix_cache == "on", kv_fp8=args.kv_dtype == "fp8")
 
     def barrier():
         if world > 1:
@@ -531,20 +544,24 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": sh.dtype,
+            "vs_baseline": None, "dtype": "fp8_e4m3 cache, " + sh.dtype if rep.kv_fp8 else sh.dtype,
             "data": "synthetic (seeded counter-based K/V/q values; seeded lengths, pool order and stops)",
             "config": {"workload": describe(args.workload), "n_seqs": rep.n, "num_layers": rep.NL,
                        "block_size": sh.block_size, "num_q_heads": sh.num_q_heads,
                        "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim, "split_tokens": args.split,
                        "parallelism": f"replicas x{world}",
+                       "kv_cache": ("E4M3 codes + one power-of-two scale byte per (token, KV head) row"
+                                    if rep.kv_fp8 else sh.dtype),
                        "l2": "no flush: the KV read per step exceeds the 126 MB L2"},
             "decode_tokens_per_s": round(world * rep.n * K / (ms * 1e-3), 1),
             "kv_gb_per_step": round(kv_tot / K / 1e9 / world, 4),
             "hbm_fraction_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
-                         "traffic": captured_traffic() if args.workload == "continuous_batch" else None,
-                         "kernel": "paged_decode_mma_kernel (+ split_reduce_kernel)",
+                         "traffic": (captured_traffic() if args.workload == "continuous_batch" and not rep.kv_fp8
+                                     else None),
+                         "kernel": ("fp8::decode_kernel" if rep.kv_fp8 else "paged_decode_mma_kernel")
+                                   + " (+ split_reduce_kernel)",
                          "attn_ms_mean": round(attn_mean_ms, 4), "alg_bytes_per_launch": int(alg_per_launch),
                          "launches_timed": len(attn_ms), "peak_source": peak_src},
             "gpu_launches": int(launches),
@@ -562,7 +579,7 @@ def run_ours(args):
             line["e2e"] = {"value": round(e2e_kv / (e2e_ms * 1e-3) / 1e9, 1), "unit": UNIT,
                            "h2d_bytes_per_step": int(e2e_io[0]), "d2h_bytes_per_step": int(e2e_io[1]),
                            "ms_per_step": round(e2e_ms / K, 4)}
-        if not args.no_cpu_baseline and args.workload not in ("prefix_sharing", "shared_prompt"):
+        if not args.no_cpu_baseline and args.workload not in ("prefix_sharing", "shared_prompt") and not rep.kv_fp8:
             line["cpu_baseline"] = cpu_baseline(rep, args.cpu_sample_seqs, W, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if world > 1:

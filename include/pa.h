@@ -53,7 +53,8 @@ typedef enum {
     PA_ERR_UNSUPPORTED = 5     /* a valid shape the kernels are not built for */
 } pa_status;
 
-typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+/* PA_FP8_E4M3 is a cache storage type only: see "FP8 cache" below. */
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_FP8_E4M3 = 3 } pa_dtype;
 
 typedef struct pa_pool pa_pool;
 typedef void *pa_stream;       /* a cudaStream_t */
@@ -65,6 +66,9 @@ typedef struct {
     int32_t num_kv_heads;      /* >= 1 */
     int32_t head_dim;          /* 64 or 128 */
     pa_dtype dtype;            /* element type of the K and V pools */
+    pa_dtype act_dtype;        /* PA_FP8_E4M3 pools: type of queries, appended rows and
+                                  16-bit outputs (PA_F16 or PA_BF16); ignored otherwise
+                                  (they are the pool dtype) */
 } pa_pool_config;
 
 typedef struct {
@@ -85,6 +89,26 @@ typedef struct {
 const char *pa_last_error(void);
 const char *pa_status_string(pa_status s);
 
+/* ------------------------------------------------------------------ FP8 cache
+ *
+ * [P1] "Common misconception": paging does not shrink the bytes each token needs;
+ * KV-cache quantisation does.  A pool of dtype PA_FP8_E4M3 stores every key and
+ * value element as one E4M3 byte (OCP 8-bit floating point, "fn" variant: bias 7,
+ * 3 mantissa bits, largest finite 448, 0x7F / 0xFF NaN) and, beside the codes, one
+ * scale byte per (token, KV head) row of K and of V in one caller-owned device array
+ *   scales [num_layers][num_blocks][num_kv_heads][2][block_size] uint8
+ * (index 0 = K, 1 = V), byte e meaning the factor 2^(e - 127).  A row x of head_dim
+ * values is written by pa_append_kv as: X = the smallest integer with
+ * max|x| <= 448 * 2^X, clamped to [-127, 127] (an all-zero row gets -127);
+ * e = X + 127; code_i = x_i * 2^-X (one fp32 multiply) rounded to nearest E4M3,
+ * ties to even, saturating at 448.
+ * Readers use the value E4M3(code) * 2^(e - 127).  The scales are per row, so an
+ * append never re-encodes earlier rows of its block, and copy-on-write, swap and
+ * decode carry them with the codes.  Non-finite input rows are outside the
+ * contract.  Supported: decode (head_dim 128), append, block copies and swap;
+ * pa_prefill_attention returns PA_ERR_UNSUPPORTED for FP8 pools.
+ */
+
 /* ------------------------------------------------------------------ pool */
 
 /* Create the host block manager for caller-owned device pools.
@@ -97,6 +121,10 @@ pa_status pa_pool_create(const pa_pool_config *cfg, void *k_pool, void *v_pool,
                          const int32_t *free_order, pa_pool **out);
 pa_status pa_pool_destroy(pa_pool *pool);
 pa_status pa_pool_stats(const pa_pool *pool, pa_pool_stats_t *out);
+/* Attach the scale array of a PA_FP8_E4M3 pool (device, 16-byte aligned,
+ * caller-owned, layout above).  Required before any device call on such a pool;
+ * PA_ERR_INVALID_ARG for other pools or a null pointer. */
+pa_status pa_pool_set_scales(pa_pool *pool, void *scales);
 
 /* ------------------------------------------------------------------ blocks */
 
@@ -196,7 +224,9 @@ pa_status pa_prefix_evictable(const pa_pool *pool, int32_t *out, int32_t cap, in
  * sequence's cache to host memory and bring it back.
  * Host buffer layout (caller-owned, page-locked so the GPU can reach it, e.g. from
  * cudaHostAlloc): [block i in logical order][layer][K, V][num_kv_heads][block_size]
- * [head_dim] of the pool dtype; pa_swap_bytes gives its size. */
+ * [head_dim] of the pool dtype; for a PA_FP8_E4M3 pool each [block][layer] record
+ * is followed by the block's scale bytes [num_kv_heads][2][block_size].
+ * pa_swap_bytes gives the size. */
 pa_status pa_swap_bytes(const pa_pool *pool, int32_t seq_id, size_t *bytes);
 /* Enqueue on `stream` a copy of every block of seq_id (all layers, K and V) into
  * host_buf, then drop one reference on each block (logical order), as a retire does.
@@ -214,7 +244,8 @@ pa_status pa_swap_in(pa_pool *pool, int32_t seq_id, const void *host_buf, size_t
 
 /* Copy-on-write block copies: for each pair (src, dst) in pairs_dev[n_pairs][2]
  * (device int32), block dst becomes a bit copy of block src in every layer, keys
- * and values.  The whole block is copied, so every earlier slot stays valid. */
+ * and values (and their scale bytes in an FP8 pool).  The whole block is copied,
+ * so every earlier slot stays valid. */
 pa_status pa_copy_blocks(pa_pool *pool, const int32_t *pairs_dev, int32_t n_pairs,
                          pa_stream stream);
 
@@ -222,7 +253,8 @@ pa_status pa_copy_blocks(pa_pool *pool, const int32_t *pairs_dev, int32_t n_pair
  * [num_kv_heads][head_dim] of the pool dtype, 16-byte aligned) is bit-copied
  * into slot slot_mapping_dev[i] of `layer`; a negative slot skips the row
  * ([P1] "Why the KV cache becomes the problem": decode appends a small amount
- * of new data each step). */
+ * of new data each step).  For a PA_FP8_E4M3 pool the rows are of act_dtype and
+ * each (token, head) row is quantised as stated under "FP8 cache". */
 pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const void *v_new,
                        const int64_t *slot_mapping_dev, int32_t n_tokens, pa_stream stream);
 
@@ -239,15 +271,16 @@ size_t pa_decode_workspace_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t he
  * head g = h / (num_q_heads / num_kv_heads) and L = seq_lens_dev[s]:
  *   out[s][h] = sum_{j<L} softmax_j(scale * q[s][h] . K_s[j]) V_s[j],
  *   K_s[j] = k_pool[layer][tables[s][j / B]][g][j % B], V_s likewise.
- * q [n_seqs][num_q_heads][head_dim] in the pool dtype; out the same shape in
- * out_dtype (PA_F32 or the pool dtype); block_tables_dev [n_seqs][max_blocks]
+ * q [n_seqs][num_q_heads][head_dim] in the pool dtype (act_dtype for an FP8
+ * pool, whose K_s[j] / V_s[j] are the dequantised rows); out the same shape in
+ * out_dtype (PA_F32 or the pool dtype / act_dtype); block_tables_dev [n_seqs][max_blocks]
  * int32, seq_lens_dev [n_seqs] int32 >= 1, all device pointers.  Sequences with
  * more than split_tokens tokens (a multiple of block_size; 0 = never) are split
  * into ranges of split_tokens, each reduced by a second kernel; that needs
  * `workspace` of pa_decode_workspace_bytes(n_seqs, num_q_heads, head_dim,
  * pa_decode_max_splits(...)) bytes (caller-owned device memory, 16-byte aligned,
- * contents need not be initialised).  Supported: head_dim 64/128, block_size
- * 16/32, num_q_heads / num_kv_heads in {1, 2, 4, 8}. */
+ * contents need not be initialised).  Supported: head_dim 64/128 (128 for FP8
+ * pools), block_size 16/32, num_q_heads / num_kv_heads in {1, 2, 4, 8}. */
 pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void *out,
                               pa_dtype out_dtype, const int32_t *block_tables_dev,
                               int32_t max_blocks, const int32_t *seq_lens_dev, int32_t n_seqs,

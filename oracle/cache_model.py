@@ -16,10 +16,11 @@ way the pages describe:
 Writes are bit copies, so the GPU pools must match these arrays exactly.
 
 FP8 pools (``dtype == "fp8"``) hold E4M3 codes and, beside them, one scale byte per
-(token, KV head) row in arrays [num_layers][num_blocks][num_kv_heads][block_size];
-an appended row is quantised by ``oracle.fp8.quantize_rows`` (the format and the
-scale rule are stated there), and block copies and swaps carry the scales with the
-codes.
+(token, KV head) row of K and of V, in one array [num_layers][num_blocks][num_kv_heads]
+[2][block_size] (index 0 = K, 1 = V; a layout reading: a block's scales for one head
+sit together, next to those of the neighbouring heads); an appended row is quantised
+by ``oracle.fp8.quantize_rows`` (the format and the scale rule are stated there), and
+block copies and swaps carry the scales with the codes.
 """
 from __future__ import annotations
 
@@ -41,12 +42,11 @@ def empty_pools(num_layers, num_blocks, num_kv_heads, block_size, head_dim, dtyp
 
 
 def empty_scales(num_layers, num_blocks, num_kv_heads, block_size):
-    """Scale-byte arrays of an FP8 pool (K and V), [layers][blocks][kv heads][block_size]."""
-    shape = (num_layers, num_blocks, num_kv_heads, block_size)
-    return np.zeros(shape, np.uint8), np.zeros(shape, np.uint8)
+    """Scale bytes of an FP8 pool, [layers][blocks][kv heads][K, V][block_size]."""
+    return np.zeros((num_layers, num_blocks, num_kv_heads, 2, block_size), np.uint8)
 
 
-def append_rows_fp8(k_pool, v_pool, k_scales, v_scales, layer, slots, k_rows, v_rows, act_dtype):
+def append_rows_fp8(k_pool, v_pool, scales, layer, slots, k_rows, v_rows, act_dtype):
     """Quantise row i of k_rows / v_rows ([n][Hkv][d], storage of ``act_dtype``) and
     write its codes and scale bytes into slot slots[i] of ``layer``."""
     from . import widen                      # the oracle's own exact decoders
@@ -60,8 +60,8 @@ def append_rows_fp8(k_pool, v_pool, k_scales, v_scales, layer, slots, k_rows, v_
         blk, off = divmod(slot, block_size)
         k_pool[layer, blk, :, off, :] = kc[i]
         v_pool[layer, blk, :, off, :] = vc[i]
-        k_scales[layer, blk, :, off] = ks[i]
-        v_scales[layer, blk, :, off] = vs[i]
+        scales[layer, blk, :, 0, off] = ks[i]
+        scales[layer, blk, :, 1, off] = vs[i]
 
 
 def append_rows(k_pool, v_pool, layer, slots, k_rows, v_rows):
@@ -83,33 +83,31 @@ def copy_blocks(k_pool, v_pool, pairs):
         v_pool[:, int(dst)] = v_pool[:, int(src)]
 
 
-def copy_scales(k_scales, v_scales, pairs):
+def copy_scales(scales, pairs):
     """The scale bytes travel with a copied FP8 block, every layer."""
     for src, dst in pairs:
-        k_scales[:, int(dst)] = k_scales[:, int(src)]
-        v_scales[:, int(dst)] = v_scales[:, int(src)]
+        scales[:, int(dst)] = scales[:, int(src)]
 
 
-def swap_buffer_fp8(k_pool, v_pool, k_scales, v_scales, blocks):
+def swap_buffer_fp8(k_pool, v_pool, scales, blocks):
     """Host copy of a swapped-out sequence of an FP8 pool, as bytes: for block i in
     logical order and each layer, the K codes [heads][block_size][dim], the V codes,
-    then the K scale bytes [heads][block_size] and the V scale bytes (reading: the
-    scales ride in the same block-major record as their codes)."""
+    then the block's scale bytes [heads][K, V][block_size] (reading: the scales ride in
+    the same block-major record as their codes)."""
     out = []
     for b in blocks:
         for layer in range(k_pool.shape[0]):
-            out += [k_pool[layer, int(b)].ravel(), v_pool[layer, int(b)].ravel(),
-                    k_scales[layer, int(b)].ravel(), v_scales[layer, int(b)].ravel()]
+            out += [k_pool[layer, int(b)].ravel(), v_pool[layer, int(b)].ravel(), scales[layer, int(b)].ravel()]
     return np.concatenate(out) if out else np.zeros(0, np.uint8)
 
 
-def swap_restore_fp8(k_pool, v_pool, k_scales, v_scales, blocks, buf):
+def swap_restore_fp8(k_pool, v_pool, scales, blocks, buf):
     nl, _, h, bs, d = k_pool.shape
     pos = 0
     for b in blocks:
         for layer in range(nl):
             for arr, n, shape in ((k_pool, h * bs * d, (h, bs, d)), (v_pool, h * bs * d, (h, bs, d)),
-                                  (k_scales, h * bs, (h, bs)), (v_scales, h * bs, (h, bs))):
+                                  (scales, 2 * h * bs, (h, 2, bs))):
                 arr[layer, int(b)] = buf[pos:pos + n].reshape(shape)
                 pos += n
 

@@ -15,8 +15,8 @@ from . import _native
 from ._native import PoolConfig, PoolStats
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_OUT_OF_BLOCKS, PA_ERR_DOUBLE_FREE, PA_ERR_CUDA, PA_ERR_UNSUPPORTED = range(6)
-PA_F32, PA_F16, PA_BF16 = 0, 1, 2
-DTYPE_CODES = {"f32": PA_F32, "f16": PA_F16, "bf16": PA_BF16}
+PA_F32, PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2, 3
+DTYPE_CODES = {"f32": PA_F32, "f16": PA_F16, "bf16": PA_BF16, "fp8": PA_FP8_E4M3}
 
 
 class PaError(RuntimeError):
@@ -71,9 +71,11 @@ def _stream(stream):
 
 # ------------------------------------------------------------------ pool
 def pa_pool_create(num_layers, num_blocks, block_size, num_kv_heads, head_dim, dtype,
-                   k_pool=None, v_pool=None, free_order=None):
-    """Host block manager over caller-owned device pools (None for host-only use)."""
-    cfg = PoolConfig(num_layers, num_blocks, block_size, num_kv_heads, head_dim, _dtype_code(dtype))
+                   k_pool=None, v_pool=None, free_order=None, act_dtype=None):
+    """Host block manager over caller-owned device pools (None for host-only use).
+    ``act_dtype`` is the query / appended-row type of an "fp8" pool."""
+    act = _dtype_code(act_dtype) if act_dtype is not None else _dtype_code(dtype)
+    cfg = PoolConfig(num_layers, num_blocks, block_size, num_kv_heads, head_dim, _dtype_code(dtype), act)
     order = None
     if free_order is not None:
         order = np.ascontiguousarray(free_order, dtype=np.int32)
@@ -81,6 +83,11 @@ def pa_pool_create(num_layers, num_blocks, block_size, num_kv_heads, head_dim, d
     _check(_lib().pa_pool_create(ctypes.byref(cfg), _dev_ptr(k_pool), _dev_ptr(v_pool),
                                  _host_ptr(order), ctypes.byref(out)))
     return out
+
+
+def pa_pool_set_scales(pool, scales) -> None:
+    """Attach the uint8 scale array [layers][blocks][kv heads][K, V][block_size] of an FP8 pool."""
+    _check(_lib().pa_pool_set_scales(pool, _dev_ptr(scales)))
 
 
 def pa_pool_destroy(pool) -> None:

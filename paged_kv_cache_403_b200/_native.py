@@ -15,7 +15,8 @@ P_i32 = ctypes.POINTER(c_i32)
 
 class PoolConfig(ctypes.Structure):
     _fields_ = [("num_layers", c_i32), ("num_blocks", c_i32), ("block_size", c_i32),
-                ("num_kv_heads", c_i32), ("head_dim", c_i32), ("dtype", ctypes.c_int)]
+                ("num_kv_heads", c_i32), ("head_dim", c_i32), ("dtype", ctypes.c_int),
+                ("act_dtype", ctypes.c_int)]
 
 
 class PoolStats(ctypes.Structure):
@@ -32,6 +33,7 @@ SIGNATURES = {
     "pa_pool_create": (ctypes.c_int, [ctypes.POINTER(PoolConfig), c_vp, c_vp, c_vp, ctypes.POINTER(c_vp)]),
     "pa_pool_destroy": (ctypes.c_int, [c_vp]),
     "pa_pool_stats": (ctypes.c_int, [c_vp, ctypes.POINTER(PoolStats)]),
+    "pa_pool_set_scales": (ctypes.c_int, [c_vp, c_vp]),
     "pa_alloc_block": (ctypes.c_int, [c_vp, P_i32]),
     "pa_free_block": (ctypes.c_int, [c_vp, c_i32]),
     "pa_incref_block": (ctypes.c_int, [c_vp, c_i32]),

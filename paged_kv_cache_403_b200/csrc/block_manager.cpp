@@ -153,8 +153,12 @@ pa_status pa_pool_create(const pa_pool_config *cfg, void *k_pool, void *v_pool,
     if (cfg->num_layers < 1 || cfg->num_blocks < 1 || cfg->num_kv_heads < 1 ||
         cfg->block_size < 1 || cfg->head_dim < 1)
         return fail(PA_ERR_INVALID_ARG, "pa_pool_create: sizes must be positive");
-    if (cfg->dtype != PA_F32 && cfg->dtype != PA_F16 && cfg->dtype != PA_BF16)
+    if (cfg->dtype != PA_F32 && cfg->dtype != PA_F16 && cfg->dtype != PA_BF16 && cfg->dtype != PA_FP8_E4M3)
         return fail(PA_ERR_INVALID_ARG, "pa_pool_create: unknown dtype");
+    if (cfg->dtype == PA_FP8_E4M3 && cfg->act_dtype != PA_F16 && cfg->act_dtype != PA_BF16)
+        return fail(PA_ERR_INVALID_ARG, "pa_pool_create: an FP8 pool needs act_dtype PA_F16 or PA_BF16");
+    if (cfg->dtype == PA_FP8_E4M3 && cfg->block_size % 16 != 0)
+        return fail(PA_ERR_UNSUPPORTED, "pa_pool_create: FP8 pools need a block_size that is a multiple of 16");
     if ((k_pool == nullptr) != (v_pool == nullptr))
         return fail(PA_ERR_INVALID_ARG, "pa_pool_create: give both pools or neither");
     if (((uintptr_t)k_pool | (uintptr_t)v_pool) & 15)
@@ -187,6 +191,14 @@ pa_status pa_pool_create(const pa_pool_config *cfg, void *k_pool, void *v_pool,
         for (int32_t i = 0; i < nb; ++i) p->free_stack[nb - 1 - i] = i;
     }
     *out = p;
+    return PA_OK;
+}
+
+pa_status pa_pool_set_scales(pa_pool *pool, void *scales) {
+    if (!pool || !scales) return fail(PA_ERR_INVALID_ARG, "pa_pool_set_scales: null argument");
+    if (!pool->fp8()) return fail(PA_ERR_INVALID_ARG, "pa_pool_set_scales: only FP8 pools carry scales");
+    if ((uintptr_t)scales & 15) return fail(PA_ERR_INVALID_ARG, "pa_pool_set_scales: scales must be 16-byte aligned");
+    pool->scales = scales;
     return PA_OK;
 }
 
@@ -483,7 +495,7 @@ pa_status pa_prefix_evictable(const pa_pool *p, int32_t *out, int32_t cap, int32
 
 static size_t swap_bytes_of(const pa_pool *p, int32_t len) {
     const size_t nblk = (size_t)((len + p->cfg.block_size - 1) / p->cfg.block_size);
-    return nblk * (size_t)p->cfg.num_layers * 2 * p->block_bytes();
+    return nblk * (size_t)p->cfg.num_layers * p->swap_record_bytes();
 }
 
 pa_status pa_swap_bytes(const pa_pool *p, int32_t seq_id, size_t *bytes) {

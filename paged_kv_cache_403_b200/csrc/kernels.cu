@@ -12,6 +12,8 @@
 //                          decode appends a small amount of new data).
 //  copy_blocks_kernel   -- copy-on-write block copies (same page, "How
 //                          PagedAttention works").
+//  paged_decode_mma_kernel (below), prefill.cuh and fp8.cuh hold the tensor-core
+//  decode, the tcgen05 chunked prefill and the FP8-cache append and decode.
 //
 // Design (B200): each (block, KV head) tile of keys or values is one contiguous
 // block_size x head_dim run in HBM, fetched whole by a 1-D TMA bulk copy
@@ -30,6 +32,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <string>
@@ -879,6 +882,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) paged_decode_mma_kernel(con
 }
 
 #include "prefill.cuh"
+#include "fp8.cuh"
 
 // ------------------------------------------------------------------ append / copy
 struct AppendParams {
@@ -916,9 +920,11 @@ __global__ void __launch_bounds__(128) append_kv_kernel(const AppendParams p) {
 struct CopyParams {
     unsigned char *k_pool;
     unsigned char *v_pool;
+    unsigned char *scales;    // FP8 pools: scale bytes (null otherwise)
     const int32_t *pairs;     // [n][2] (src, dst)
     int64_t block_chunks;     // 16-byte chunks per block (all heads)
     int64_t layer_chunks;     // 16-byte chunks per layer
+    int64_t scale_block_chunks, scale_layer_chunks;
     int32_t num_blocks;
 };
 
@@ -935,6 +941,11 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p) {
     uint4 *from = pool + layer * p.layer_chunks + (int64_t)src * p.block_chunks;
     uint4 *to = pool + layer * p.layer_chunks + (int64_t)dst * p.block_chunks;
     for (int64_t t = threadIdx.x; t < p.block_chunks; t += blockDim.x) to[t] = from[t];
+    if (p.scales && blockIdx.z == 0) {
+        uint4 *sc = reinterpret_cast<uint4 *>(p.scales) + layer * p.scale_layer_chunks;
+        for (int64_t t = threadIdx.x; t < p.scale_block_chunks; t += blockDim.x)
+            sc[(int64_t)dst * p.scale_block_chunks + t] = sc[(int64_t)src * p.scale_block_chunks + t];
+    }
 }
 
 // ------------------------------------------------------------------ swap copies
@@ -943,9 +954,12 @@ constexpr int kSwapChunk = 256;   // block ids passed by value per launch
 struct SwapParams {
     unsigned char *k_pool;
     unsigned char *v_pool;
+    unsigned char *scales;        // FP8 pools: scale bytes (null otherwise)
     unsigned char *host;          // device-visible address of the page-locked host buffer
     int64_t block_chunks;         // 16-byte chunks of one block (all heads) in one layer
     int64_t layer_chunks;         // 16-byte chunks of one layer of the pool
+    int64_t scale_block_chunks, scale_layer_chunks;
+    int64_t record_chunks;        // one [block][layer] record of the host buffer
     int32_t num_blocks, first, count, to_host;
     int32_t blocks[kSwapChunk];
 };
@@ -963,12 +977,20 @@ __global__ void __launch_bounds__(256) swap_copy_kernel(const __grid_constant__ 
     uint4 *pool = reinterpret_cast<uint4 *>(kv == 0 ? p.k_pool : p.v_pool) + layer * p.layer_chunks +
                   (int64_t)blk * p.block_chunks;
     const int64_t layers = gridDim.y;
-    uint4 *host = reinterpret_cast<uint4 *>(p.host) +
-                  (((int64_t)(p.first + i) * layers + layer) * 2 + kv) * p.block_chunks;
+    uint4 *rec = reinterpret_cast<uint4 *>(p.host) + ((int64_t)(p.first + i) * layers + layer) * p.record_chunks;
+    uint4 *host = rec + kv * p.block_chunks;
     if (p.to_host)
         for (int64_t t = threadIdx.x; t < p.block_chunks; t += blockDim.x) host[t] = pool[t];
     else
         for (int64_t t = threadIdx.x; t < p.block_chunks; t += blockDim.x) pool[t] = host[t];
+    if (p.scales && kv == 0) {
+        uint4 *sc = reinterpret_cast<uint4 *>(p.scales) + layer * p.scale_layer_chunks + (int64_t)blk * p.scale_block_chunks;
+        uint4 *hs = rec + 2 * p.block_chunks;
+        if (p.to_host)
+            for (int64_t t = threadIdx.x; t < p.scale_block_chunks; t += blockDim.x) hs[t] = sc[t];
+        else
+            for (int64_t t = threadIdx.x; t < p.scale_block_chunks; t += blockDim.x) sc[t] = hs[t];
+    }
 }
 
 // ------------------------------------------------------------------ host dispatch
@@ -1057,10 +1079,25 @@ pa_status dispatch_mma(const MmaParams &p, const ReduceParams &r, int n_seqs, in
     return fail(PA_ERR_UNSUPPORTED, "block_size must be 16 or 32 and head_dim 64 or 128");
 }
 
-// TMA descriptors over a 16-bit pool: 2-D [rows][head_dim], boxes of 64 elements
-// (128 bytes, the 128-byte swizzle span) by block_size rows.
-pa_status ensure_tensor_maps(pa_pool *pool) {
-    if (pool->tmaps_ready) return PA_OK;
+template <typename T, int B, int HEADS>
+pa_status launch_fp8(const fp8::Params &p, const ReduceParams &r, int n_seqs, cudaStream_t stream) {
+    constexpr size_t smem = fp8::Shape<B, HEADS>::kSmemBytes;
+    auto kernel = fp8::decode_kernel<T, B, HEADS>;
+    static bool smem_set[64] = {};
+    pa_status st = ensure_smem(kernel, smem, smem_set);
+    if (st != PA_OK) return st;
+    dim3 grid(n_seqs, p.num_kv_heads / HEADS, p.max_splits);
+    kernel<<<grid, kDecodeThreads, smem, stream>>>(p);
+    pa_internal::launch_count.fetch_add(1);
+    st = check_launch("fp8::decode_kernel");
+    if (st != PA_OK) return st;
+    return launch_reduce<T, B, fp8::kD>(r, n_seqs, stream);
+}
+
+// TMA descriptors over a 16-bit or FP8 pool: 2-D [rows][head_dim], boxes of 128
+// bytes (the 128-byte swizzle span: 64 16-bit elements or 128 codes) by block_size rows.
+pa_status ensure_tensor_maps(pa_pool *pool, int box_rows) {
+    if (pool->tmaps_ready && pool->tmap_rows == box_rows) return PA_OK;
     using Encode = PFN_cuTensorMapEncodeTiled_v12000;
     static Encode encode = nullptr;
     if (!encode) {
@@ -1075,10 +1112,13 @@ pa_status ensure_tensor_maps(pa_pool *pool) {
     const uint64_t rows = (uint64_t)c.num_layers * c.num_blocks * c.num_kv_heads * c.block_size;
     if (rows >= (1ull << 31))
         return fail(PA_ERR_UNSUPPORTED, "pool too large for 32-bit TMA row coordinates");
-    const CUtensorMapDataType dt = c.dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const CUtensorMapDataType dt = c.dtype == PA_BF16       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : c.dtype == PA_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const size_t eb = pool->elem_bytes();
     cuuint64_t dims[2] = {(cuuint64_t)c.head_dim, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)c.head_dim * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)c.block_size};
+    cuuint64_t strides[1] = {(cuuint64_t)(c.head_dim * eb)};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / eb), (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     void *bases[2] = {pool->k_pool, pool->v_pool};
     CUtensorMap *maps[2] = {&pool->tmap_k, &pool->tmap_v};
@@ -1089,6 +1129,7 @@ pa_status ensure_tensor_maps(pa_pool *pool) {
         if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")");
     }
     pool->tmaps_ready = true;
+    pool->tmap_rows = box_rows;
     return PA_OK;
 }
 
@@ -1160,7 +1201,8 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
                               const int32_t *block_tables_dev, int32_t max_blocks, const int32_t *seq_lens_dev,
                               int32_t n_seqs, int32_t num_q_heads, float scale, int32_t split_tokens,
                               void *workspace, size_t ws_bytes, pa_stream stream) {
-    if (!pool || !pool->k_pool) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: pool has no device memory");
+    if (!pool || !pool->device_ready())
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: pool has no device memory (or no FP8 scales)");
     const pa_pool_config &c = pool->cfg;
     if (layer < 0 || layer >= c.num_layers) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: layer out of range");
     if (n_seqs < 0 || max_blocks < 1) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: bad n_seqs/max_blocks");
@@ -1169,8 +1211,10 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
         return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: null device pointer");
     if (!aligned16(q) || !aligned16(out) || ((uintptr_t)block_tables_dev & 3) || ((uintptr_t)seq_lens_dev & 3))
         return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: misaligned pointer");
-    if (out_dtype != PA_F32 && out_dtype != c.dtype)
-        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: out_dtype must be PA_F32 or the pool dtype");
+    if (out_dtype != PA_F32 && out_dtype != pool->act_dtype())
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: out_dtype must be PA_F32 or the pool's query type");
+    if (pool->fp8() && c.head_dim != fp8::kD)
+        return fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: FP8 pools need head_dim 128");
     if (num_q_heads < 1 || num_q_heads % c.num_kv_heads != 0)
         return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: num_q_heads must be a multiple of num_kv_heads");
     const int group = num_q_heads / c.num_kv_heads;
@@ -1228,7 +1272,46 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
         const int hpc = group < 4 ? group : 4;
         return dispatch_simt<float>(p, r, c.block_size, c.head_dim, hpc, st);
     }
-    pa_status s2 = ensure_tensor_maps(pool);
+    if (pool->fp8()) {
+        const int heads = fp8::heads_per_cta(group, c.num_kv_heads, c.block_size);
+        pa_status s2 = ensure_tensor_maps(pool, heads * c.block_size);
+        if (s2 != PA_OK) return s2;
+        fp8::Params p;
+        p.tmap_k = pool->tmap_k;
+        p.tmap_v = pool->tmap_v;
+        p.s_layer = static_cast<const unsigned char *>(pool->scales) + (size_t)layer * pool->scale_layer_bytes();
+        p.q = q;
+        p.out = out;
+        p.tables = block_tables_dev;
+        p.lens = seq_lens_dev;
+        p.ws_acc = ws_acc;
+        p.ws_ml = ws_ml;
+        p.max_blocks = max_blocks;
+        p.num_blocks = c.num_blocks;
+        p.num_kv_heads = c.num_kv_heads;
+        p.num_q_heads = num_q_heads;
+        p.layer = layer;
+        p.split_blocks = split_blocks;
+        p.max_splits = max_splits;
+        p.out_f32 = r.out_f32;
+        p.group = group;
+        p.scale_log2 = scale_log2;
+        const bool bf = c.act_dtype == PA_BF16;
+#define PA_FP8_LAUNCH(B, H) \
+    (bf ? launch_fp8<__nv_bfloat16, B, H>(p, r, n_seqs, st) : launch_fp8<__half, B, H>(p, r, n_seqs, st))
+        if (c.block_size == 16) {
+            if (heads == 4) return PA_FP8_LAUNCH(16, 4);
+            if (heads == 2) return PA_FP8_LAUNCH(16, 2);
+            return PA_FP8_LAUNCH(16, 1);
+        }
+        if (c.block_size == 32) {
+            if (heads == 2) return PA_FP8_LAUNCH(32, 2);
+            return PA_FP8_LAUNCH(32, 1);
+        }
+#undef PA_FP8_LAUNCH
+        return fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: block_size must be 16 or 32");
+    }
+    pa_status s2 = ensure_tensor_maps(pool, c.block_size);
     if (s2 != PA_OK) return s2;
     MmaParams p;
     p.tmap_k = pool->tmap_k;
@@ -1268,7 +1351,7 @@ pa_status pa_prefill_attention(pa_pool *pool, int32_t layer, const void *q, void
     if (!aligned16(q) || !aligned16(out) || ((uintptr_t)block_tables_dev & 3) || ((uintptr_t)seq_lens_dev & 3) ||
         ((uintptr_t)q_start_dev & 3))
         return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: misaligned pointer");
-    if (c.dtype == PA_F32)
+    if (c.dtype == PA_F32 || c.dtype == PA_FP8_E4M3)
         return fail(PA_ERR_UNSUPPORTED, "pa_prefill_attention: the tensor-core path takes fp16 / bf16 caches");
     if (c.head_dim != 128 || (c.block_size != 16 && c.block_size != 32))
         return fail(PA_ERR_UNSUPPORTED, "pa_prefill_attention: head_dim 128 and block_size 16 or 32 only");
@@ -1284,7 +1367,7 @@ pa_status pa_prefill_attention(pa_pool *pool, int32_t layer, const void *q, void
                           (prefill::kTiles * prefill::kRows);
     if (tiles > INT32_MAX || c.num_kv_heads > 65535 || n_seqs > 65535)
         return fail(PA_ERR_UNSUPPORTED, "pa_prefill_attention: grid too large");
-    pa_status st = ensure_tensor_maps(pool);
+    pa_status st = ensure_tensor_maps(pool, c.block_size);
     if (st != PA_OK) return st;
     prefill::Params p;
     p.tmap_k = pool->tmap_k;
@@ -1312,13 +1395,47 @@ pa_status pa_prefill_attention(pa_pool *pool, int32_t layer, const void *q, void
 
 pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const void *v_new,
                        const int64_t *slot_mapping_dev, int32_t n_tokens, pa_stream stream) {
-    if (!pool || !pool->k_pool) return fail(PA_ERR_INVALID_ARG, "pa_append_kv: pool has no device memory");
+    if (!pool || !pool->device_ready())
+        return fail(PA_ERR_INVALID_ARG, "pa_append_kv: pool has no device memory (or no FP8 scales)");
     if (layer < 0 || layer >= pool->cfg.num_layers) return fail(PA_ERR_INVALID_ARG, "pa_append_kv: layer out of range");
     if (n_tokens < 0) return fail(PA_ERR_INVALID_ARG, "pa_append_kv: negative n_tokens");
     if (n_tokens == 0) return PA_OK;
     if (!k_new || !v_new || !slot_mapping_dev || !aligned16(k_new) || !aligned16(v_new) ||
         ((uintptr_t)slot_mapping_dev & 7))
         return fail(PA_ERR_INVALID_ARG, "pa_append_kv: null or misaligned device pointer");
+    if (pool->fp8()) {
+        const pa_pool_config &c = pool->cfg;
+        if (c.head_dim != 64 && c.head_dim != 128)
+            return fail(PA_ERR_UNSUPPORTED, "pa_append_kv: FP8 pools need head_dim 64 or 128");
+        fp8::AppendParams p;
+        p.k_layer = static_cast<unsigned char *>(pool->k_pool) + (size_t)layer * pool->layer_bytes();
+        p.v_layer = static_cast<unsigned char *>(pool->v_pool) + (size_t)layer * pool->layer_bytes();
+        p.s_layer = static_cast<unsigned char *>(pool->scales) + (size_t)layer * pool->scale_layer_bytes();
+        p.k_new = static_cast<const unsigned char *>(k_new);
+        p.v_new = static_cast<const unsigned char *>(v_new);
+        p.slots = slot_mapping_dev;
+        p.n_tokens = n_tokens;
+        p.block_size = c.block_size;
+        p.num_kv_heads = c.num_kv_heads;
+        p.num_blocks = c.num_blocks;
+        const int64_t warps = 2 * (int64_t)n_tokens * c.num_kv_heads;
+        const int grid = (int)std::min<int64_t>((warps + 7) / 8, 148 * 16);
+        cudaStream_t cs = static_cast<cudaStream_t>(stream);
+        const bool bf = c.act_dtype == PA_BF16;
+        if (c.head_dim == 128) {
+            if (bf)
+                fp8::append_kernel<__nv_bfloat16, 128><<<grid, 256, 0, cs>>>(p);
+            else
+                fp8::append_kernel<__half, 128><<<grid, 256, 0, cs>>>(p);
+        } else {
+            if (bf)
+                fp8::append_kernel<__nv_bfloat16, 64><<<grid, 256, 0, cs>>>(p);
+            else
+                fp8::append_kernel<__half, 64><<<grid, 256, 0, cs>>>(p);
+        }
+        pa_internal::launch_count.fetch_add(1);
+        return check_launch("fp8::append_kernel");
+    }
     const size_t row_bytes = (size_t)pool->cfg.head_dim * pool->elem_bytes();
     if (row_bytes % 16) return fail(PA_ERR_UNSUPPORTED, "pa_append_kv: head_dim * element size must be a multiple of 16");
     AppendParams p;
@@ -1339,7 +1456,8 @@ pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const vo
 }
 
 pa_status pa_copy_blocks(pa_pool *pool, const int32_t *pairs_dev, int32_t n_pairs, pa_stream stream) {
-    if (!pool || !pool->k_pool) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: pool has no device memory");
+    if (!pool || !pool->device_ready())
+        return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: pool has no device memory (or no FP8 scales)");
     if (n_pairs < 0) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: negative n_pairs");
     if (n_pairs == 0) return PA_OK;
     if (!pairs_dev || ((uintptr_t)pairs_dev & 3)) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: bad pairs pointer");
@@ -1348,9 +1466,12 @@ pa_status pa_copy_blocks(pa_pool *pool, const int32_t *pairs_dev, int32_t n_pair
     CopyParams p;
     p.k_pool = static_cast<unsigned char *>(pool->k_pool);
     p.v_pool = static_cast<unsigned char *>(pool->v_pool);
+    p.scales = static_cast<unsigned char *>(pool->scales);
     p.pairs = pairs_dev;
     p.block_chunks = (int64_t)(pool->block_bytes() / 16);
     p.layer_chunks = (int64_t)(pool->layer_bytes() / 16);
+    p.scale_block_chunks = (int64_t)(pool->scale_block_bytes() / 16);
+    p.scale_layer_chunks = (int64_t)(pool->scale_layer_bytes() / 16);
     p.num_blocks = pool->cfg.num_blocks;
     copy_blocks_kernel<<<dim3(n_pairs, pool->cfg.num_layers, 2), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
     pa_internal::launch_count.fetch_add(1);
@@ -1414,13 +1535,18 @@ pa_status swap_copy(const pa_pool *pool, const int32_t *blocks, int32_t n, void 
     }
     if (((uintptr_t)attr.devicePointer & 15) || pool->block_bytes() % 16)
         return fail(PA_ERR_INVALID_ARG, "swap: host buffer must be 16-byte aligned");
+    if (!pool->device_ready()) return fail(PA_ERR_INVALID_ARG, "swap: the FP8 pool has no scale arrays");
     if (pool->cfg.num_layers > 65535) return fail(PA_ERR_UNSUPPORTED, "swap: too many layers");
     SwapParams p;
     p.k_pool = static_cast<unsigned char *>(pool->k_pool);
     p.v_pool = static_cast<unsigned char *>(pool->v_pool);
+    p.scales = static_cast<unsigned char *>(pool->scales);
     p.host = static_cast<unsigned char *>(attr.devicePointer);
     p.block_chunks = (int64_t)(pool->block_bytes() / 16);
     p.layer_chunks = (int64_t)(pool->layer_bytes() / 16);
+    p.scale_block_chunks = (int64_t)(pool->scale_block_bytes() / 16);
+    p.scale_layer_chunks = (int64_t)(pool->scale_layer_bytes() / 16);
+    p.record_chunks = (int64_t)(pool->swap_record_bytes() / 16);
     p.num_blocks = pool->cfg.num_blocks;
     p.to_host = to_host ? 1 : 0;
     for (int32_t first = 0; first < n; first += kSwapChunk) {

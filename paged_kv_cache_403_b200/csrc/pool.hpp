@@ -15,6 +15,7 @@ struct pa_pool {
     pa_pool_config cfg;
     void *k_pool = nullptr;   // device, [L][NB][Hkv][B][D]
     void *v_pool = nullptr;
+    void *scales = nullptr;   // FP8 pools: device scale bytes [L][NB][Hkv][K, V][B]
 
     // Free list: a LIFO stack; back() is handed out next.
     std::vector<int32_t> free_stack;
@@ -49,10 +50,21 @@ struct pa_pool {
     // [num_layers * num_blocks * num_kv_heads * block_size rows][head_dim]; built on
     // the first decode call (16-bit caches only).
     bool tmaps_ready = false;
+    int tmap_rows = 0;                // box height of the cached descriptors
     CUtensorMap tmap_k;
     CUtensorMap tmap_v;
 
-    size_t elem_bytes() const { return cfg.dtype == PA_F32 ? 4 : 2; }
+    bool fp8() const { return cfg.dtype == PA_FP8_E4M3; }
+    // type of queries, appended rows and 16-bit outputs
+    pa_dtype act_dtype() const { return fp8() ? cfg.act_dtype : cfg.dtype; }
+    size_t elem_bytes() const { return cfg.dtype == PA_F32 ? 4 : fp8() ? 1 : 2; }
+    size_t act_bytes() const { return act_dtype() == PA_F32 ? 4 : 2; }
+    // FP8 pools: scale bytes of one block (all heads, K and V) in one layer, and of a layer
+    size_t scale_block_bytes() const { return fp8() ? (size_t)2 * cfg.num_kv_heads * cfg.block_size : 0; }
+    size_t scale_layer_bytes() const { return scale_block_bytes() * (size_t)cfg.num_blocks; }
+    // one [block][layer] record of a swap buffer: K codes, V codes, then the scales
+    size_t swap_record_bytes() const { return 2 * block_bytes() + scale_block_bytes(); }
+    bool device_ready() const { return k_pool && (!fp8() || scales); }
     // bytes of one (block, kv-head) tile and of one block across heads
     size_t tile_bytes() const { return (size_t)cfg.block_size * cfg.head_dim * elem_bytes(); }
     size_t block_bytes() const { return tile_bytes() * cfg.num_kv_heads; }
@@ -65,7 +77,8 @@ pa_status fail(pa_status st, const std::string &msg);
 pa_status ok();
 extern std::atomic<uint64_t> launch_count;
 // Device side of swapping (kernels.cu): copy `blocks` between the pools and a host
-// buffer laid out [block][layer][K, V][Hkv][B][D]; to_host selects the direction.
+// buffer of [block][layer] records (K codes, V codes, then for FP8 pools the block's
+// scale bytes); to_host selects the direction.
 pa_status swap_copy(const pa_pool *pool, const int32_t *blocks, int32_t n, void *host_buf, bool to_host,
                     void *stream);
 }  // namespace pa_internal

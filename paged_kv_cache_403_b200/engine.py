@@ -18,30 +18,40 @@ import torch
 
 from . import (pa_append_kv, pa_build_block_tables, pa_copy_blocks, pa_decode_attention,
                pa_decode_max_splits, pa_decode_workspace_bytes, pa_pool_create, pa_pool_destroy,
-               pa_pool_stats, pa_reserve_slots, pa_seq_add, pa_seq_fork, pa_seq_free, pa_seq_info)
+               pa_pool_set_scales, pa_pool_stats, pa_reserve_slots, pa_seq_add, pa_seq_fork, pa_seq_free,
+               pa_seq_info)
 
-TORCH_DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+TORCH_DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16, "fp8": torch.uint8}
 
 
 class PagedCache:
     def __init__(self, num_layers, num_blocks, block_size, num_kv_heads, head_dim, dtype,
-                 free_order=None, device="cuda"):
+                 free_order=None, device="cuda", act_dtype=None):
+        """``dtype`` "fp8" stores E4M3 codes plus per-row scale bytes; ``act_dtype`` ("f16" or
+        "bf16") is then the type of queries, appended rows and 16-bit outputs."""
         self.num_layers, self.num_blocks, self.block_size = num_layers, num_blocks, block_size
         self.num_kv_heads, self.head_dim, self.dtype = num_kv_heads, head_dim, dtype
+        self.act_dtype = act_dtype if dtype == "fp8" else dtype
         self.device = device
+        self.scales = None
         if device is not None:
             shape = (num_layers, num_blocks, num_kv_heads, block_size, head_dim)
             self.k_pool = torch.zeros(shape, dtype=TORCH_DTYPES[dtype], device=device)
             self.v_pool = torch.zeros(shape, dtype=TORCH_DTYPES[dtype], device=device)
+            if dtype == "fp8":
+                self.scales = torch.zeros((num_layers, num_blocks, num_kv_heads, 2, block_size), dtype=torch.uint8,
+                                          device=device)
         else:
             self.k_pool = self.v_pool = None
         self.pool = pa_pool_create(num_layers, num_blocks, block_size, num_kv_heads, head_dim, dtype,
-                                   self.k_pool, self.v_pool, free_order)
+                                   self.k_pool, self.v_pool, free_order, self.act_dtype)
+        if self.scales is not None:
+            pa_pool_set_scales(self.pool, self.scales)
 
     @classmethod
     def from_shape(cls, shape, free_order=None, device="cuda"):
         return cls(shape.num_layers, shape.num_blocks, shape.block_size, shape.num_kv_heads,
-                   shape.head_dim, shape.dtype, free_order, device)
+                   shape.head_dim, shape.dtype, free_order, device, getattr(shape, "act_dtype", None))
 
     def close(self):
         if self.pool is not None:

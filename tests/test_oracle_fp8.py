@@ -189,23 +189,24 @@ def test_cache_model_append_and_copy_fp8():
     from oracle import cache_model as cm
     rng = np.random.default_rng(7)
     kp, vp = cm.empty_pools(2, 6, 2, 16, 64, "fp8")
-    ksc, vsc = cm.empty_scales(2, 6, 2, 16)
+    sc = cm.empty_scales(2, 6, 2, 16)
     rows_k = rng.standard_normal((3, 2, 64)).astype(np.float16)
     rows_v = rng.standard_normal((3, 2, 64)).astype(np.float16)
-    cm.append_rows_fp8(kp, vp, ksc, vsc, 1, [5 * 16 + 3, -1, 2 * 16], rows_k, rows_v, "f16")
-    codes, sc = FP8.quantize_rows(rows_k.astype(np.float32))
-    assert np.array_equal(kp[1, 5, :, 3], codes[0]) and np.array_equal(ksc[1, 5, :, 3], sc[0])
-    assert np.array_equal(kp[1, 2, :, 0], codes[2])
-    assert kp[0].sum() == 0 and np.count_nonzero(ksc) == 4      # two rows x two heads, layer 1 only
+    cm.append_rows_fp8(kp, vp, sc, 1, [5 * 16 + 3, -1, 2 * 16], rows_k, rows_v, "f16")
+    codes, ks = FP8.quantize_rows(rows_k.astype(np.float32))
+    _, vs = FP8.quantize_rows(rows_v.astype(np.float32))
+    assert np.array_equal(kp[1, 5, :, 3], codes[0]) and np.array_equal(sc[1, 5, :, 0, 3], ks[0])
+    assert np.array_equal(sc[1, 5, :, 1, 3], vs[0]) and np.array_equal(kp[1, 2, :, 0], codes[2])
+    assert kp[0].sum() == 0 and np.count_nonzero(sc) == 8       # 2 rows x 2 heads x K, V; layer 1 only
     cm.copy_blocks(kp, vp, [(5, 1)])
-    cm.copy_scales(ksc, vsc, [(5, 1)])
-    assert np.array_equal(kp[:, 1], kp[:, 5]) and np.array_equal(vsc[:, 1], vsc[:, 5])
-    buf = cm.swap_buffer_fp8(kp, vp, ksc, vsc, [5, 2])
+    cm.copy_scales(sc, [(5, 1)])
+    assert np.array_equal(kp[:, 1], kp[:, 5]) and np.array_equal(sc[:, 1], sc[:, 5])
+    buf = cm.swap_buffer_fp8(kp, vp, sc, [5, 2])
     assert buf.size == 2 * 2 * (2 * 2 * 16 * 64 + 2 * 2 * 16)
     k2, v2 = cm.empty_pools(2, 6, 2, 16, 64, "fp8")
-    ks2, vs2 = cm.empty_scales(2, 6, 2, 16)
-    cm.swap_restore_fp8(k2, v2, ks2, vs2, [0, 4], buf)
-    assert np.array_equal(k2[:, 0], kp[:, 5]) and np.array_equal(vs2[:, 4], vsc[:, 2])
+    sc2 = cm.empty_scales(2, 6, 2, 16)
+    cm.swap_restore_fp8(k2, v2, sc2, [0, 4], buf)
+    assert np.array_equal(k2[:, 0], kp[:, 5]) and np.array_equal(sc2[:, 4], sc[:, 2])
 
 
 def test_bytes_per_token_halved_for_the_pages_model():
