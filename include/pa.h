@@ -261,7 +261,9 @@ pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const vo
 /* Number of splits per sequence the decode kernel uses for a table of width
  * max_blocks when a split holds split_tokens tokens (0 = never split). */
 int32_t pa_decode_max_splits(int32_t block_size, int32_t max_blocks, int32_t split_tokens);
-/* Workspace bytes pa_decode_attention needs for that many splits (0 if 1). */
+/* Workspace bytes for pa_decode_attention with that many splits: the split partials
+ * (when max_splits > 1) plus the longest-first order of the (sequence, split)
+ * ranges, int32 [n_seqs * max_splits], each rounded up to 16 bytes. */
 size_t pa_decode_workspace_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t head_dim,
                                  int32_t max_splits);
 
@@ -279,7 +281,10 @@ size_t pa_decode_workspace_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t he
  * into ranges of split_tokens, each reduced by a second kernel; that needs
  * `workspace` of pa_decode_workspace_bytes(n_seqs, num_q_heads, head_dim,
  * pa_decode_max_splits(...)) bytes (caller-owned device memory, 16-byte aligned,
- * contents need not be initialised).  Supported: head_dim 64/128 (128 for FP8
+ * contents need not be initialised).  With a workspace of that size the call first
+ * sorts the ranges by length on the device (one small kernel) and starts the longest
+ * ranges first, so no long range is left running alone at the end; with a single
+ * split the workspace may be NULL, and the ranges then start in batch order.  Supported: head_dim 64/128 (128 for FP8
  * pools), block_size 16/32, num_q_heads / num_kv_heads in {1, 2, 4, 8}. */
 pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void *out,
                               pa_dtype out_dtype, const int32_t *block_tables_dev,

@@ -150,8 +150,9 @@ struct Params {
     const int32_t *lens;
     float *ws_acc;
     float *ws_ml;
+    const int32_t *order;           // longest-first range order, or null (launch order)
     int32_t max_blocks, num_blocks, num_kv_heads, num_q_heads, layer;
-    int32_t split_blocks, max_splits, out_f32, group;
+    int32_t split_blocks, max_splits, out_f32, group, head_groups;
     float scale_log2;
 };
 
@@ -181,16 +182,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
 
-    const int s = blockIdx.x;
-    const int g0 = blockIdx.y * HEADS;      // first KV head of this CTA
-    const int split = blockIdx.z;
+    // one CTA per (range, head group); ranges longest first when an order is given
+    const int hg = (int)(blockIdx.x % (unsigned)p.head_groups);
+    const int rank = (int)(blockIdx.x / (unsigned)p.head_groups);
+    const int item = p.order ? p.order[rank] : rank;
+    const int s = item / p.max_splits;
+    const int split = item % p.max_splits;
+    const int g0 = hg * HEADS;              // first KV head of this CTA
     const int group = p.group;
     const int hpc = HEADS * group;          // query heads of this CTA (<= 8)
     const int h0 = g0 * group;
 
     int L = p.lens[s];
     if (L < 1 || (L + B - 1) / B > p.max_blocks) {
-        if (threadIdx.x == 0 && blockIdx.y == 0 && split == 0) raise_error(kErrBadLen);
+        if (threadIdx.x == 0 && hg == 0 && split == 0) raise_error(kErrBadLen);
         if (L < 1) {
             if (split == 0)
                 for (int t = threadIdx.x; t < hpc * kD; t += blockDim.x) {

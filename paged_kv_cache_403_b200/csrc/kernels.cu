@@ -515,6 +515,77 @@ __global__ void __launch_bounds__(D) split_reduce_kernel(const ReduceParams p) {
         static_cast<T *>(p.out)[idx] = Elem<T>::narrow(v);
 }
 
+// ------------------------------------------------------------------ longest ranges first
+// The decode grid has one CTA per (sequence, split range, head group), and ranges range
+// from a few tokens to a whole split.  The block scheduler starts CTAs in index order,
+// so a long range that starts late keeps a few SMs busy after the rest are idle.  One
+// CTA of this kernel sorts the (sequence, split) ranges by tile count, longest first
+// (a counting sort over the counts), and the decode kernels take their range from
+// that order: the greedy longest-first schedule.  Ranges of equal length may come in
+// any order; each range's result is the same wherever it runs.
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBuckets = 4096;   // counts >= 4095 tiles share the first bucket
+
+struct PlanParams {
+    const int32_t *lens;
+    int32_t *order;                  // [n_seqs * max_splits] range ids s * max_splits + z
+    int32_t n_seqs, max_blocks, block_size, split_blocks, max_splits;
+};
+
+__device__ __forceinline__ int plan_bucket(const PlanParams &p, int item) {
+    const int s = item / p.max_splits, z = item % p.max_splits;
+    const int L = p.lens[s];
+    const int nblk = L < 1 ? 0 : min((L + p.block_size - 1) / p.block_size, p.max_blocks);
+    const int t = max(0, min(p.split_blocks, nblk - z * p.split_blocks));
+    return kPlanBuckets - 1 - min(t, kPlanBuckets - 1);   // longest ranges in the lowest bucket
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) {
+    __shared__ int start[kPlanBuckets];
+    __shared__ int warp_sum[kPlanThreads / 32];
+    constexpr int PER = kPlanBuckets / kPlanThreads;
+    const int n_items = p.n_seqs * p.max_splits;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int b = threadIdx.x; b < kPlanBuckets; b += kPlanThreads) start[b] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_items; i += kPlanThreads) atomicAdd(&start[plan_bucket(p, i)], 1);
+    __syncthreads();
+    // exclusive prefix sum of the bucket counts: PER buckets per thread, then warps
+    int cnt[PER], sum = 0;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        cnt[k] = start[threadIdx.x * PER + k];
+        sum += cnt[k];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int w = warp_sum[lane];
+        int wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi += v;
+        }
+        warp_sum[lane] = wi - w;
+    }
+    __syncthreads();
+    int run = warp_sum[warp] + incl - sum;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        start[threadIdx.x * PER + k] = run;
+        run += cnt[k];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_items; i += kPlanThreads) p.order[atomicAdd(&start[plan_bucket(p, i)], 1)] = i;
+}
+
 // ------------------------------------------------------------------ tensor-core decode (fp16 / bf16)
 // Per consumer warp and per 16-token group of a tile:
 //   S^T[16 tok][8 heads]  = K[16][D] . Q^T[D][8]       mma.m16n8k16, K rows via ldmatrix
@@ -606,8 +677,9 @@ struct MmaParams {
     const int32_t *lens;
     float *ws_acc;
     float *ws_ml;
+    const int32_t *order;           // longest-first range order, or null (launch order)
     int32_t max_blocks, num_blocks, num_kv_heads, num_q_heads, layer;
-    int32_t split_blocks, max_splits, out_f32, heads_per_cta;
+    int32_t split_blocks, max_splits, out_f32, heads_per_cta, head_groups;
     float scale_log2;
 };
 
@@ -633,9 +705,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) paged_decode_mma_kernel(con
     // 128-byte swizzled TMA destinations want 1024-byte alignment
     unsigned char *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
 
-    const int s = blockIdx.x;
-    const int hg = blockIdx.y;
-    const int split = blockIdx.z;
+    // one CTA per (range, head group); ranges longest first when an order is given
+    const int hg = (int)(blockIdx.x % (unsigned)p.head_groups);
+    const int rank = (int)(blockIdx.x / (unsigned)p.head_groups);
+    const int item = p.order ? p.order[rank] : rank;
+    const int s = item / p.max_splits;
+    const int split = item % p.max_splits;
     const int hpc = p.heads_per_cta;
 
     int L = p.lens[s];
@@ -1062,7 +1137,7 @@ pa_status launch_mma(const MmaParams &p, const ReduceParams &r, int n_seqs, cuda
     static bool smem_set[64] = {};
     pa_status st = ensure_smem(kernel, smem, smem_set);
     if (st != PA_OK) return st;
-    dim3 grid(n_seqs, p.num_q_heads / p.heads_per_cta, p.max_splits);
+    const dim3 grid((unsigned)((int64_t)n_seqs * p.max_splits * p.head_groups));
     kernel<<<grid, kDecodeThreads, smem, stream>>>(p);
     pa_internal::launch_count.fetch_add(1);
     st = check_launch("paged_decode_mma_kernel");
@@ -1086,7 +1161,7 @@ pa_status launch_fp8(const fp8::Params &p, const ReduceParams &r, int n_seqs, cu
     static bool smem_set[64] = {};
     pa_status st = ensure_smem(kernel, smem, smem_set);
     if (st != PA_OK) return st;
-    dim3 grid(n_seqs, p.num_kv_heads / HEADS, p.max_splits);
+    const dim3 grid((unsigned)((int64_t)n_seqs * p.max_splits * p.head_groups));
     kernel<<<grid, kDecodeThreads, smem, stream>>>(p);
     pa_internal::launch_count.fetch_add(1);
     st = check_launch("fp8::decode_kernel");
@@ -1148,6 +1223,19 @@ pa_status launch_prefill(const prefill::Params &p, dim3 grid, cudaStream_t strea
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Decode workspace: split partials (acc [parts][D] then (m, l) [parts][2], fp32) when a
+// sequence can have more than one split, then the longest-first range order
+// (int32 [n_seqs * max_splits]), each part rounded up to 16 bytes.
+size_t partial_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_splits) {
+    if (max_splits <= 1) return 0;
+    const size_t parts = (size_t)n_seqs * max_splits * num_q_heads;
+    return (parts * head_dim * sizeof(float) + parts * 2 * sizeof(float) + 15) & ~(size_t)15;
+}
+
+size_t order_bytes(int32_t n_seqs, int32_t max_splits) {
+    return ((size_t)n_seqs * max_splits * sizeof(int32_t) + 15) & ~(size_t)15;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ allocation-free decode
@@ -1192,9 +1280,8 @@ int32_t pa_decode_max_splits(int32_t block_size, int32_t max_blocks, int32_t spl
 }
 
 size_t pa_decode_workspace_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_splits) {
-    if (n_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_splits <= 1) return 0;
-    const size_t parts = (size_t)n_seqs * max_splits * num_q_heads;
-    return parts * head_dim * sizeof(float) + parts * 2 * sizeof(float);
+    if (n_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_splits < 1) return 0;
+    return partial_bytes(n_seqs, num_q_heads, head_dim, max_splits) + order_bytes(n_seqs, max_splits);
 }
 
 pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void *out, pa_dtype out_dtype,
@@ -1226,16 +1313,44 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
     const int32_t max_splits = pa_decode_max_splits(c.block_size, max_blocks, split_tokens);
     if (max_splits > 65535 || num_q_heads > 65535)
         return fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: grid too large");
+    const size_t need_partials = partial_bytes(n_seqs, num_q_heads, c.head_dim, max_splits);
     const size_t need = pa_decode_workspace_bytes(n_seqs, num_q_heads, c.head_dim, max_splits);
-    if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
-        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: workspace missing, misaligned or smaller than " +
+    if (workspace && !aligned16(workspace))
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: workspace must be 16-byte aligned");
+    if (need_partials > 0 && (!workspace || ws_bytes < need_partials))
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: workspace missing or smaller than " +
                                             std::to_string(need) + " bytes");
 
     const size_t parts = (size_t)n_seqs * max_splits * num_q_heads;
     float *ws_acc = static_cast<float *>(workspace);
-    float *ws_ml = need > 0 ? static_cast<float *>(workspace) + parts * c.head_dim : nullptr;
+    float *ws_ml = need_partials > 0 ? static_cast<float *>(workspace) + parts * c.head_dim : nullptr;
     const int32_t split_blocks = split_tokens > 0 ? split_tokens / c.block_size : max_blocks;
     const float scale_log2 = (float)((double)scale * 1.4426950408889634);   // scale * log2(e)
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // Longest ranges first, when the workspace has room for the order and the grid is
+    // more than about two CTAs per SM (below that there is no tail to shape).
+    const int head_groups = c.dtype == PA_F32 ? 0
+                            : pool->fp8() ? c.num_kv_heads / fp8::heads_per_cta(group, c.num_kv_heads, c.block_size)
+                                          : c.num_kv_heads;
+    if ((int64_t)n_seqs * max_splits * (head_groups > 0 ? head_groups : 1) >= (1ll << 31))
+        return fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: grid too large");
+    int32_t *order = nullptr;
+    if (head_groups > 0 && workspace && ws_bytes >= need &&
+        (int64_t)n_seqs * max_splits * head_groups > 2 * 148) {
+        order = reinterpret_cast<int32_t *>(static_cast<unsigned char *>(workspace) + need_partials);
+        PlanParams pp;
+        pp.lens = seq_lens_dev;
+        pp.order = order;
+        pp.n_seqs = n_seqs;
+        pp.max_blocks = max_blocks;
+        pp.block_size = c.block_size;
+        pp.split_blocks = split_blocks;
+        pp.max_splits = max_splits;
+        plan_kernel<<<1, kPlanThreads, 0, st>>>(pp);
+        pa_internal::launch_count.fetch_add(1);
+        pa_status ps = check_launch("plan_kernel");
+        if (ps != PA_OK) return ps;
+    }
 
     ReduceParams r;
     r.lens = seq_lens_dev;
@@ -1248,7 +1363,6 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
     r.max_splits = max_splits;
     r.out_f32 = out_dtype == PA_F32;
 
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (c.dtype == PA_F32) {
         // fp32 caches: CUDA-core kernel (the tensor-core path takes 16-bit operands only)
         DecodeParams p;
@@ -1295,6 +1409,8 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
         p.max_splits = max_splits;
         p.out_f32 = r.out_f32;
         p.group = group;
+        p.head_groups = head_groups;
+        p.order = order;
         p.scale_log2 = scale_log2;
         const bool bf = c.act_dtype == PA_BF16;
 #define PA_FP8_LAUNCH(B, H) \
@@ -1331,6 +1447,8 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
     p.max_splits = max_splits;
     p.out_f32 = r.out_f32;
     p.heads_per_cta = group;   // the whole GQA group (<= 8) shares one CTA
+    p.head_groups = head_groups;
+    p.order = order;
     p.scale_log2 = scale_log2;
     if (c.dtype == PA_BF16) return dispatch_mma<__nv_bfloat16>(p, r, n_seqs, c.block_size, c.head_dim, st);
     return dispatch_mma<__half>(p, r, n_seqs, c.block_size, c.head_dim, st);
