@@ -262,8 +262,9 @@ pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const vo
  * max_blocks when a split holds split_tokens tokens (0 = never split). */
 int32_t pa_decode_max_splits(int32_t block_size, int32_t max_blocks, int32_t split_tokens);
 /* Workspace bytes for pa_decode_attention with that many splits: the split partials
- * (when max_splits > 1) plus the longest-first order of the (sequence, split)
- * ranges, int32 [n_seqs * max_splits], each rounded up to 16 bytes. */
+ * (when max_splits > 1), the longest-first order of the (sequence, split) ranges
+ * (int32 [n_seqs * max_splits]) and, with splits, one merge counter per (sequence,
+ * query head) at most; each part rounded up to 16 bytes. */
 size_t pa_decode_workspace_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t head_dim,
                                  int32_t max_splits);
 
@@ -278,7 +279,8 @@ size_t pa_decode_workspace_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t he
  * out_dtype (PA_F32 or the pool dtype / act_dtype); block_tables_dev [n_seqs][max_blocks]
  * int32, seq_lens_dev [n_seqs] int32 >= 1, all device pointers.  Sequences with
  * more than split_tokens tokens (a multiple of block_size; 0 = never) are split
- * into ranges of split_tokens, each reduced by a second kernel; that needs
+ * into ranges of split_tokens whose partial results are merged (on the tensor-core
+ * paths by the last CTA of each range, on the fp32 path by a second kernel); that needs
  * `workspace` of pa_decode_workspace_bytes(n_seqs, num_q_heads, head_dim,
  * pa_decode_max_splits(...)) bytes (caller-owned device memory, 16-byte aligned,
  * contents need not be initialised).  With a workspace of that size the call first

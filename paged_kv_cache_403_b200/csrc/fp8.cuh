@@ -151,6 +151,7 @@ struct Params {
     float *ws_acc;
     float *ws_ml;
     const int32_t *order;           // longest-first range order, or null (launch order)
+    int32_t *counters;              // [n_seqs][head_groups] split-merge counters
     int32_t max_blocks, num_blocks, num_kv_heads, num_q_heads, layer;
     int32_t split_blocks, max_splits, out_f32, group, head_groups;
     float scale_log2;
@@ -520,6 +521,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
                 p.ws_ml[part * 2 + 1] = lsum;
             }
         }
+    }
+    if (nsplit > 1) {
+        // (the range is looked up again rather than kept in registers across the loop)
+        const int hg2 = (int)(blockIdx.x % (unsigned)p.head_groups);
+        const int rank2 = (int)(blockIdx.x / (unsigned)p.head_groups);
+        const int s2 = (p.order ? p.order[rank2] : rank2) / p.max_splits;
+        merge_splits_if_last<T>(p.ws_acc, p.ws_ml, p.counters + (size_t)s2 * p.head_groups + hg2, p.out, p.out_f32,
+                                s2, p.num_q_heads, p.max_splits, nsplit, hg2 * HEADS * p.group, HEADS * p.group, kD);
     }
 }
 

@@ -529,7 +529,8 @@ constexpr int kPlanBuckets = 4096;   // counts >= 4095 tiles share the first buc
 struct PlanParams {
     const int32_t *lens;
     int32_t *order;                  // [n_seqs * max_splits] range ids s * max_splits + z
-    int32_t n_seqs, max_blocks, block_size, split_blocks, max_splits;
+    int32_t *counters;               // [n_counters] split-merge counters to zero
+    int32_t n_seqs, max_blocks, block_size, split_blocks, max_splits, n_counters;
 };
 
 __device__ __forceinline__ int plan_bucket(const PlanParams &p, int item) {
@@ -546,6 +547,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
     constexpr int PER = kPlanBuckets / kPlanThreads;
     const int n_items = p.n_seqs * p.max_splits;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < p.n_counters; i += kPlanThreads) p.counters[i] = 0;
     for (int b = threadIdx.x; b < kPlanBuckets; b += kPlanThreads) start[b] = 0;
     __syncthreads();
     for (int i = threadIdx.x; i < n_items; i += kPlanThreads) atomicAdd(&start[plan_bucket(p, i)], 1);
@@ -584,6 +586,50 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
     }
     __syncthreads();
     for (int i = threadIdx.x; i < n_items; i += kPlanThreads) p.order[atomicAdd(&start[plan_bucket(p, i)], 1)] = i;
+}
+
+// ------------------------------------------------------------------ in-kernel split merge
+// The tensor-core decode kernels merge split partials themselves: every split CTA of a
+// (sequence, head group) writes its partial, fences, and bumps that range's counter;
+// the CTA that brings the counter to the number of splits merges all partials of its
+// query heads (the same log-sum-exp merge as split_reduce_kernel) and writes the
+// output, then resets the counter.  The counters are zeroed by plan_kernel, which
+// runs before every split launch.  This saves the reduce launch and its re-read of
+// cold partials (the last CTA finds most of them in L2).
+template <typename T>
+__device__ __forceinline__ void merge_splits_if_last(const float *ws_acc, const float *ws_ml, int32_t *counter,
+                                                     void *out, int out_f32, int s, int num_q_heads,
+                                                     int max_splits, int nsplit, int h0, int hpc, int D) {
+    __shared__ int is_last;
+    __threadfence();          // this CTA's partial is visible before the count moves
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int prev = atomicAdd(counter, 1);
+        is_last = prev == nsplit - 1;
+        if (is_last) *counter = 0;
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (int t = threadIdx.x; t < hpc * D; t += blockDim.x) {
+        const int h = t / D;
+        const int d = t % D;
+        const size_t base = (size_t)s * max_splits * num_q_heads + h0 + h;
+        float mx = -INFINITY;
+        for (int x = 0; x < nsplit; ++x) mx = fmaxf(mx, __ldcg(ws_ml + (base + (size_t)x * num_q_heads) * 2));
+        float lsum = 0.f, osum = 0.f;
+        for (int x = 0; x < nsplit; ++x) {
+            const size_t part = base + (size_t)x * num_q_heads;
+            const float f = ex2(__ldcg(ws_ml + part * 2) - mx);
+            lsum += __ldcg(ws_ml + part * 2 + 1) * f;
+            osum += __ldcg(ws_acc + part * D + d) * f;
+        }
+        const size_t idx = ((size_t)s * num_q_heads + h0 + h) * D + d;
+        if (out_f32)
+            static_cast<float *>(out)[idx] = osum / lsum;
+        else
+            static_cast<T *>(out)[idx] = Elem<T>::narrow(osum / lsum);
+    }
 }
 
 // ------------------------------------------------------------------ tensor-core decode (fp16 / bf16)
@@ -678,6 +724,7 @@ struct MmaParams {
     float *ws_acc;
     float *ws_ml;
     const int32_t *order;           // longest-first range order, or null (launch order)
+    int32_t *counters;              // [n_seqs][head_groups] split-merge counters
     int32_t max_blocks, num_blocks, num_kv_heads, num_q_heads, layer;
     int32_t split_blocks, max_splits, out_f32, heads_per_cta, head_groups;
     float scale_log2;
@@ -954,6 +1001,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) paged_decode_mma_kernel(con
             }
         }
     }
+    if (nsplit > 1)
+        merge_splits_if_last<T>(p.ws_acc, p.ws_ml, p.counters + (size_t)s * p.head_groups + hg, p.out, p.out_f32, s,
+                                p.num_q_heads, p.max_splits, nsplit, h0, hpc, D);
 }
 
 #include "prefill.cuh"
@@ -1140,9 +1190,7 @@ pa_status launch_mma(const MmaParams &p, const ReduceParams &r, int n_seqs, cuda
     const dim3 grid((unsigned)((int64_t)n_seqs * p.max_splits * p.head_groups));
     kernel<<<grid, kDecodeThreads, smem, stream>>>(p);
     pa_internal::launch_count.fetch_add(1);
-    st = check_launch("paged_decode_mma_kernel");
-    if (st != PA_OK) return st;
-    return launch_reduce<T, B, D>(r, n_seqs, stream);
+    return check_launch("paged_decode_mma_kernel");   // splits are merged in the kernel
 }
 
 template <typename T>
@@ -1164,9 +1212,7 @@ pa_status launch_fp8(const fp8::Params &p, const ReduceParams &r, int n_seqs, cu
     const dim3 grid((unsigned)((int64_t)n_seqs * p.max_splits * p.head_groups));
     kernel<<<grid, kDecodeThreads, smem, stream>>>(p);
     pa_internal::launch_count.fetch_add(1);
-    st = check_launch("fp8::decode_kernel");
-    if (st != PA_OK) return st;
-    return launch_reduce<T, B, fp8::kD>(r, n_seqs, stream);
+    return check_launch("fp8::decode_kernel");   // splits are merged in the kernel
 }
 
 // TMA descriptors over a 16-bit or FP8 pool: 2-D [rows][head_dim], boxes of 128
@@ -1236,6 +1282,12 @@ size_t order_bytes(int32_t n_seqs, int32_t max_splits) {
     return ((size_t)n_seqs * max_splits * sizeof(int32_t) + 15) & ~(size_t)15;
 }
 
+// split-merge counters, one per (sequence, head group) -- at most num_q_heads groups
+size_t counter_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t max_splits) {
+    if (max_splits <= 1) return 0;
+    return ((size_t)n_seqs * num_q_heads * sizeof(int32_t) + 15) & ~(size_t)15;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ allocation-free decode
@@ -1281,7 +1333,8 @@ int32_t pa_decode_max_splits(int32_t block_size, int32_t max_blocks, int32_t spl
 
 size_t pa_decode_workspace_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_splits) {
     if (n_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_splits < 1) return 0;
-    return partial_bytes(n_seqs, num_q_heads, head_dim, max_splits) + order_bytes(n_seqs, max_splits);
+    return partial_bytes(n_seqs, num_q_heads, head_dim, max_splits) + order_bytes(n_seqs, max_splits) +
+           counter_bytes(n_seqs, num_q_heads, max_splits);
 }
 
 pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void *out, pa_dtype out_dtype,
@@ -1334,18 +1387,30 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
                                           : c.num_kv_heads;
     if ((int64_t)n_seqs * max_splits * (head_groups > 0 ? head_groups : 1) >= (1ll << 31))
         return fail(PA_ERR_UNSUPPORTED, "pa_decode_attention: grid too large");
-    int32_t *order = nullptr;
+    // Tensor-core paths: with splits the full workspace is needed (partials, order,
+    // merge counters) and the plan kernel runs first (it zeroes the counters); without
+    // splits the order is used when there is room for it and the grid is more than
+    // about two CTAs per SM (below that there is no tail to shape).
+    if (head_groups > 0 && max_splits > 1 && ws_bytes < need)
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: workspace smaller than " + std::to_string(need) +
+                                            " bytes");
+    int32_t *order = nullptr, *counters = nullptr;
     if (head_groups > 0 && workspace && ws_bytes >= need &&
-        (int64_t)n_seqs * max_splits * head_groups > 2 * 148) {
-        order = reinterpret_cast<int32_t *>(static_cast<unsigned char *>(workspace) + need_partials);
+        (max_splits > 1 || (int64_t)n_seqs * max_splits * head_groups > 2 * 148)) {
+        unsigned char *w = static_cast<unsigned char *>(workspace);
+        order = reinterpret_cast<int32_t *>(w + need_partials);
+        counters = max_splits > 1 ? reinterpret_cast<int32_t *>(w + need_partials + order_bytes(n_seqs, max_splits))
+                                  : nullptr;
         PlanParams pp;
         pp.lens = seq_lens_dev;
         pp.order = order;
+        pp.counters = counters;
         pp.n_seqs = n_seqs;
         pp.max_blocks = max_blocks;
         pp.block_size = c.block_size;
         pp.split_blocks = split_blocks;
         pp.max_splits = max_splits;
+        pp.n_counters = counters ? n_seqs * head_groups : 0;
         plan_kernel<<<1, kPlanThreads, 0, st>>>(pp);
         pa_internal::launch_count.fetch_add(1);
         pa_status ps = check_launch("plan_kernel");
@@ -1411,6 +1476,7 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
         p.group = group;
         p.head_groups = head_groups;
         p.order = order;
+        p.counters = counters;
         p.scale_log2 = scale_log2;
         const bool bf = c.act_dtype == PA_BF16;
 #define PA_FP8_LAUNCH(B, H) \
@@ -1449,6 +1515,7 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
     p.heads_per_cta = group;   // the whole GQA group (<= 8) shares one CTA
     p.head_groups = head_groups;
     p.order = order;
+    p.counters = counters;
     p.scale_log2 = scale_log2;
     if (c.dtype == PA_BF16) return dispatch_mma<__nv_bfloat16>(p, r, n_seqs, c.block_size, c.head_dim, st);
     return dispatch_mma<__half>(p, r, n_seqs, c.block_size, c.head_dim, st);

@@ -42,10 +42,10 @@ def test_status_strings_and_sizes():
     assert pa.pa_decode_max_splits(16, 260, 0) == 1
     assert pa.pa_decode_max_splits(16, 260, 512) == 9
     assert pa.pa_decode_max_splits(16, 260, 8) == 0          # smaller than a block
-    # split partials (only with more than one split) + the longest-first range order,
-    # each rounded up to 16 bytes
+    # split partials and merge counters (only with more than one split) + the
+    # longest-first range order, each rounded up to 16 bytes
     assert pa.pa_decode_workspace_bytes(4, 32, 128, 1) == 16
-    assert pa.pa_decode_workspace_bytes(4, 32, 128, 3) == 4 * 3 * 32 * (128 + 2) * 4 + 48
+    assert pa.pa_decode_workspace_bytes(4, 32, 128, 3) == 4 * 3 * 32 * (128 + 2) * 4 + 48 + 4 * 32 * 4
 
 
 def test_device_calls_without_device_memory_fail_cleanly():
