@@ -73,20 +73,20 @@ def parse(argv=None):
     return a
 
 
-def captured_traffic():
+def captured_traffic(fp8=False):
     """DRAM bytes per launch of the decode kernel from the committed ncu summary, if the
-    kernel source is still the one that was captured (else None)."""
+    kernel sources are still the ones that were captured (else None)."""
     import hashlib
     import re
-    prof = os.path.join(ROOT, "profiles", "decode_mma_continuous_batch.md")
-    src = os.path.join(ROOT, "paged_kv_cache_403_b200", "csrc", "kernels.cu")
+    name = "decode_fp8_continuous_batch.md" if fp8 else "decode_mma_continuous_batch.md"
+    csrc = os.path.join(ROOT, "paged_kv_cache_403_b200", "csrc")
     try:
-        text = open(prof).read()
-        sha = re.search(r"kernels.cu sha256 prefix at capture: ([0-9a-f]+)", text).group(1)
+        text = open(os.path.join(ROOT, "profiles", name)).read()
         gb = float(re.search(r"traffic per launch \(read \+ write\) \| ([0-9.]+) GB", text).group(1))
+        for src, sha in re.findall(r"([a-z0-9_]+\.cuh?) sha256 prefix at capture: ([0-9a-f]+)", text):
+            if not hashlib.sha256(open(os.path.join(csrc, src), "rb").read()).hexdigest().startswith(sha):
+                return None
     except (OSError, AttributeError):
-        return None
-    if not hashlib.sha256(open(src, "rb").read()).hexdigest().startswith(sha):
         return None
     return int(gb * 1e9)
 
@@ -558,10 +558,10 @@ def run_ours(args):
             "hbm_fraction_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
-                         "traffic": (captured_traffic() if args.workload == "continuous_batch" and not rep.kv_fp8
+                         "traffic": (captured_traffic(rep.kv_fp8) if args.workload == "continuous_batch"
                                      else None),
                          "kernel": ("fp8::decode_kernel" if rep.kv_fp8 else "paged_decode_mma_kernel")
-                                   + " (+ split_reduce_kernel)",
+                                   + " (+ plan_kernel; split partials merged in the kernel)",
                          "attn_ms_mean": round(attn_mean_ms, 4), "alg_bytes_per_launch": int(alg_per_launch),
                          "launches_timed": len(attn_ms), "peak_source": peak_src},
             "gpu_launches": int(launches),
