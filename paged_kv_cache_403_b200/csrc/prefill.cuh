@@ -16,11 +16,14 @@
 //                    softmax with a lazily moved maximum (the O row is rescaled in TMEM
 //                    only when a score passes the running maximum by 2^8), P split into
 //                    a 16-bit high part and the 16-bit rounding of the remainder, both
-//                    written to shared memory in the K-major 128-byte-swizzled layout;
-//   warp 8           tensor-core issue (one lane): S_t = Q_t K^T (M=128, N=64) and
-//                    O_t += P_t V (M=128, N=head_dim, hi and lo parts) in TMEM;
+//                    written back to TMEM (tcgen05.st) as the A operand of P V;
+//   warp 8           tensor-core issue (one lane): S_t = Q_t K^T (M=128, N=64, both
+//                    operands in shared memory) and O_t += P_t V (M=128, N=head_dim,
+//                    hi and lo parts; A = P from TMEM, B = V from shared memory);
 //   warp 9           TMA producer: 64-key tiles of K and V (2-D tensor loads, 128-byte
-//                    swizzle) into a 2-stage ring, walking the block table.
+//                    swizzle) into a 4-stage ring, walking the block table.
+// P never touches shared memory, which leaves room for four K/V stages: a tile is
+// requested four tiles before the tensor core needs it.
 // The two tiles ping-pong: while one warpgroup computes exponentials the tensor core
 // works on the other tile.  Every hand-off is an mbarrier; every wait is bounded and
 // sets a shared abort flag that all roles check; TMEM is always freed.  Key rows past
@@ -35,15 +38,16 @@ constexpr int kSoftmaxThreads = kTiles * kRows;
 constexpr int kThreads = kSoftmaxThreads + 64;   // + tensor-core issue warp + TMA warp
 constexpr int kMmaWarp = kSoftmaxThreads / 32, kTmaWarp = kMmaWarp + 1;
 constexpr int kD = 128;              // head_dim
-constexpr uint32_t kTmemCols = 512;  // O_A [0,128) O_B [128,256) S_A [256,320) S_B [320,384)
-constexpr uint32_t kOCol = 0, kSCol = 256;
+// TMEM columns: O_A [0,128) O_B [128,256) S_A [256,320) S_B [320,384) P_A [384,448)
+// P_B [448,512); a P region holds the 64 keys' high halves in its first 32 columns
+// (two 16-bit values per column) and the low halves in the next 32.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kOCol = 0, kSCol = 256, kPCol = 384;
 constexpr int kQBytes = kRows * kD * 2;         // 32 KB per tile: [2 halves][128 rows][128 B]
 constexpr int kKVBytes = kKeys * kD * 2;        // 16 KB: [2 halves][64 rows][128 B]
-constexpr int kPBytes = kRows * kKeys * 2;      // 16 KB per part: [128 rows][128 B]
-constexpr int kStages = 2;
+constexpr int kStages = 4;
 constexpr int kNumBars = 3 * kTiles + 2 * kStages;
-constexpr int kSmemBytes = 1024 + kTiles * kQBytes + kStages * 2 * kKVBytes + kTiles * 2 * kPBytes +
-                           kNumBars * 8 + 16;
+constexpr int kSmemBytes = 1024 + kTiles * kQBytes + kStages * 2 * kKVBytes + kNumBars * 8 + 16;
 
 // --- tcgen05 wrappers --------------------------------------------------------------
 // Shared-memory matrix descriptor, 128-byte swizzle: start address, leading and stride
@@ -71,6 +75,16 @@ __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, ui
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// the same with A read from tensor memory (a_tmem: lane = row, two 16-bit K elements
+// per 32-bit column, 8 columns per K = 16 step)
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
 
@@ -168,8 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
     unsigned char *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     unsigned char *sQ = smem;                                       // tile t at t * kQBytes
     unsigned char *sKV = sQ + kTiles * kQBytes;                     // stage st: K then V
-    unsigned char *sP = sKV + kStages * 2 * kKVBytes;               // tile t: hi, lo
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sP + kTiles * 2 * kPBytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + kStages * 2 * kKVBytes);
     uint64_t *kv_full = bars, *kv_empty = bars + kStages;
     uint64_t *s_full = bars + 2 * kStages, *p_full = s_full + kTiles, *o_done = p_full + kTiles;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
@@ -310,14 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
         };
         auto issue_pv = [&](int t, int j) {
             if (lane == 0) {
-                const uint32_t paddr = smem_addr(sP + t * 2 * kPBytes);
+                const uint32_t pcol = tmem + kPCol + t * kKeys;
                 const uint32_t vaddr = smem_addr(sKV + (j % kStages) * 2 * kKVBytes + kKVBytes);
 #pragma unroll
                 for (int kk = 0; kk < kKeys / 16; ++kk) {
                     const uint64_t b = smem_desc(vaddr + kk * 16 * 128, kKVBytes / 2, 1024);
-                    umma(tmem + kOCol + t * kD, smem_desc(paddr + kk * 32, 16, 1024), b, IDESC_O,
-                         (j > 0 || kk > 0) ? 1u : 0u);
-                    umma(tmem + kOCol + t * kD, smem_desc(paddr + kPBytes + kk * 32, 16, 1024), b, IDESC_O, 1u);
+                    umma_ts(tmem + kOCol + t * kD, pcol + kk * 8, b, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_ts(tmem + kOCol + t * kD, pcol + kKeys / 2 + kk * 8, b, IDESC_O, 1u);
                 }
                 umma_commit(&o_done[t]);
             }
@@ -346,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
         const int kmax = row_valid ? P0 + my_t : -1;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t s_col = kSCol + qtile * kKeys, o_col = kOCol + qtile * kD;
-        unsigned char *p_hi = sP + qtile * 2 * kPBytes;
+        const uint32_t p_col = kPCol + qtile * kKeys;
         const float sl = p.scale_log2;
         float m = -INFINITY, l = 0.f;
         bool ok = tile_used;
@@ -401,26 +413,23 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                 l *= f;
                 m = tmax;
             }
-            // p = 2^(s * scale_log2 - m): one FMA and one ex2 per score (-inf -> 0)
+            // p = 2^(s * scale_log2 - m): one FMA and one ex2 per score (-inf -> 0); the
+            // high and low 16-bit parts go back to this row's TMEM lane
             const float neg_m = m == -INFINITY ? 0.f : -m;
             float lp[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t w[32], r[32];
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-                uint32_t w[4], r[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = ex2(fmaf(__uint_as_float(sv[c8 * 8 + 2 * e]), sl, neg_m));
-                    const float p1 = ex2(fmaf(__uint_as_float(sv[c8 * 8 + 2 * e + 1]), sl, neg_m));
-                    w[e] = Mma<T>::pack(p0, p1);
-                    r[e] = Mma<T>::pack(p0 - Mma<T>::low(w[e]), p1 - Mma<T>::high(w[e]));
-                    lp[e] += p0 + p1;
-                }
-                const int off = row * 128 + ((c8 ^ (row & 7)) << 4);
-                *reinterpret_cast<uint4 *>(p_hi + off) = make_uint4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<uint4 *>(p_hi + kPBytes + off) = make_uint4(r[0], r[1], r[2], r[3]);
+            for (int c = 0; c < 32; ++c) {
+                const float p0 = ex2(fmaf(__uint_as_float(sv[2 * c]), sl, neg_m));
+                const float p1 = ex2(fmaf(__uint_as_float(sv[2 * c + 1]), sl, neg_m));
+                w[c] = Mma<T>::pack(p0, p1);
+                r[c] = Mma<T>::pack(p0 - Mma<T>::low(w[c]), p1 - Mma<T>::high(w[c]));
+                lp[c & 3] += p0 + p1;
             }
+            tmem_st32(tmem + lane_base + p_col, w);
+            tmem_st32(tmem + lane_base + p_col + kKeys / 2, r);
             l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-            fence_proxy_async();
+            tmem_wait_st();
             fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[qtile]);
