@@ -14,12 +14,12 @@
 //   warps 0-3 / 4-7  softmax of tile A / B: thread = row = TMEM lane; tcgen05.ld of the
 //                    row's 64 scores, causal / length mask by select, base-2 online
 //                    softmax with a lazily moved maximum (the O row is rescaled in TMEM
-//                    only when a score passes the running maximum by 2^8), P split into
-//                    a 16-bit high part and the 16-bit rounding of the remainder, both
-//                    written back to TMEM (tcgen05.st) as the A operand of P V;
+//                    only when a score passes the running maximum by 2^8), P written
+//                    back to TMEM (tcgen05.st) as the A operand of P V: for bf16 a
+//                    truncated high part plus the rounded remainder, for fp16 once;
 //   warp 8           tensor-core issue (one lane): S_t = Q_t K^T (M=128, N=64, both
 //                    operands in shared memory) and O_t += P_t V (M=128, N=head_dim,
-//                    hi and lo parts; A = P from TMEM, B = V from shared memory);
+//                    per part of P; A = P from TMEM, B = V from shared memory);
 //   warp 9           TMA producer: 64-key tiles of K and V (2-D tensor loads, 128-byte
 //                    swizzle) into a 4-stage ring, walking the block table.
 // P never touches shared memory, which leaves room for four K/V stages: a tile is
@@ -150,16 +150,29 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// Operand format code of the instruction descriptor, and how P enters P V: bf16 P
+// keeps 8 significant bits, too few for the 2e-3 bound on peaky rows, so a bf16 P is a
+// high part (the truncation of p to bf16, taken with one byte permute) plus the bf16
+// rounding of the exact remainder (~16 bits together, two products); an fp16 P keeps 11
+// bits and enters once.
 template <typename T>
 struct Fmt;
 template <>
 struct Fmt<__half> {
     static constexpr uint32_t code = 0;
+    static constexpr bool two_parts = false;
 };
 template <>
 struct Fmt<__nv_bfloat16> {
     static constexpr uint32_t code = 1;
+    static constexpr bool two_parts = true;
 };
+
+__device__ __forceinline__ uint32_t byte_perm(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
 
 struct Params {
     CUtensorMap tmap_k;
@@ -307,15 +320,22 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             fence_after_sync();
             return true;
         };
+        // Descriptors are built once: the start address sits in the low 14 bits as
+        // addr >> 4 (shared memory < 256 KB), so moving to another tile, stage or K step
+        // is one add of offset >> 4 -- a freshly built descriptor per instruction left the
+        // issuing lane, not the tensor core, as the bottleneck.
+        const uint64_t q_desc = smem_desc(smem_addr(sQ), 16, 1024);
+        const uint64_t k_desc = smem_desc(smem_addr(sKV), 16, 1024);
+        const uint64_t v_desc = smem_desc(smem_addr(sKV + kKVBytes), kKVBytes / 2, 1024);
         auto issue_s = [&](int t, int j) {
             if (lane == 0) {
-                const uint32_t qaddr = smem_addr(sQ + t * kQBytes);
-                const uint32_t kaddr = smem_addr(sKV + (j % kStages) * 2 * kKVBytes);
+                const uint64_t qa = q_desc + (uint64_t)((t * kQBytes) >> 4);
+                const uint64_t kb = k_desc + (uint64_t)(((j % kStages) * 2 * kKVBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint64_t a = smem_desc(qaddr + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = smem_desc(kaddr + (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32, 16, 1024);
-                    umma(tmem + kSCol + t * kKeys, a, b, IDESC_S, kk > 0);
+                    const uint32_t qo = ((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4;
+                    const uint32_t ko = ((kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32) >> 4;
+                    umma(tmem + kSCol + t * kKeys, qa + qo, kb + ko, IDESC_S, kk > 0);
                 }
                 umma_commit(&s_full[t]);
             }
@@ -324,12 +344,12 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
         auto issue_pv = [&](int t, int j) {
             if (lane == 0) {
                 const uint32_t pcol = tmem + kPCol + t * kKeys;
-                const uint32_t vaddr = smem_addr(sKV + (j % kStages) * 2 * kKVBytes + kKVBytes);
+                const uint64_t vb = v_desc + (uint64_t)(((j % kStages) * 2 * kKVBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < kKeys / 16; ++kk) {
-                    const uint64_t b = smem_desc(vaddr + kk * 16 * 128, kKVBytes / 2, 1024);
+                    const uint64_t b = vb + (uint64_t)((kk * 16 * 128) >> 4);
                     umma_ts(tmem + kOCol + t * kD, pcol + kk * 8, b, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
-                    umma_ts(tmem + kOCol + t * kD, pcol + kKeys / 2 + kk * 8, b, IDESC_O, 1u);
+                    if (Fmt<T>::two_parts) umma_ts(tmem + kOCol + t * kD, pcol + kKeys / 2 + kk * 8, b, IDESC_O, 1u);
                 }
                 umma_commit(&o_done[t]);
             }
@@ -343,11 +363,12 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                 ok = wait_warp(&p_full[t], j & 1, abort_flag);   // softmax t read S_t(j), wrote P_t(j)
                 if (!ok) break;
                 fence_after_sync();
-                issue_pv(t, j);
+                // next scores first: the softmax of S_t(j+1) then runs while P_t(j) V(j) does
                 if (j + 1 < n_tiles) {
                     if (t == 0) ok = ready(j + 1);
                     if (ok) issue_s(t, j + 1);
                 }
+                if (ok) issue_pv(t, j);
             }
             if (ok && lane == 0) umma_commit(&kv_empty[j % kStages]);
             __syncwarp();
@@ -387,18 +408,28 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                 for (int c = 0; c < 64; ++c)
                     if (!(key0 + c <= kmax && key0 + c < L)) sv[c] = __float_as_uint(-INFINITY);
             }
-            float smax = -INFINITY;                 // on raw scores: scale > 0 keeps the order
+            // maximum on raw scores (scale > 0 keeps the order), as a tree of 8 chains
+            float mx8[8];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) smax = fmaxf(smax, __uint_as_float(sv[c]));
+            for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sv[e]);
+#pragma unroll
+            for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sv[c]));
+            const float smax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             const float tmax = smax * sl;
-            if (j > 0) {   // P_t(j-1) consumed and O_t settled before P_t and O_t are touched
-                ok = wait_warp(&o_done[qtile], (j - 1) & 1, abort_flag);
-                if (!ok) break;
-                fence_after_sync();
-            }
-            if (tmax > m + kRescaleThreshold) {
-                const float f = ex2(m - tmax);
+            // P_t(j-1) V(j-1) may still be running: O_t and the P_t region are only touched
+            // after it completes (the exponentials below do not need it).  The rescale
+            // decision is taken per warp (tcgen05.ld / st are warp-wide); rows that do
+            // not need it scale by 1.
+            const bool need = tmax > m + kRescaleThreshold;
+            bool settled = j == 0;
+            if (__any_sync(0xffffffffu, need)) {
+                const float f = need ? ex2(m - tmax) : 1.f;
                 if (j > 0) {
+                    ok = wait_warp(&o_done[qtile], (j - 1) & 1, abort_flag);
+                    if (!ok) break;
+                    fence_after_sync();
+                    settled = true;
 #pragma unroll
                     for (int c0 = 0; c0 < kD; c0 += 32) {
                         uint32_t o[32];
@@ -410,8 +441,10 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                     }
                     tmem_wait_st();
                 }
-                l *= f;
-                m = tmax;
+                if (need) {
+                    l *= f;
+                    m = tmax;
+                }
             }
             // p = 2^(s * scale_log2 - m): one FMA and one ex2 per score (-inf -> 0); the
             // high and low 16-bit parts go back to this row's TMEM lane
@@ -422,12 +455,24 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             for (int c = 0; c < 32; ++c) {
                 const float p0 = ex2(fmaf(__uint_as_float(sv[2 * c]), sl, neg_m));
                 const float p1 = ex2(fmaf(__uint_as_float(sv[2 * c + 1]), sl, neg_m));
-                w[c] = Mma<T>::pack(p0, p1);
-                r[c] = Mma<T>::pack(p0 - Mma<T>::low(w[c]), p1 - Mma<T>::high(w[c]));
+                if (Fmt<T>::two_parts) {
+                    // high halves of the two fp32 words = their bf16 truncations; the
+                    // remainders are exact in fp32 and rounded once to bf16
+                    const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+                    w[c] = byte_perm(b0, b1, 0x7632u);
+                    r[c] = Mma<T>::pack(p0 - __uint_as_float(b0 & 0xffff0000u), p1 - __uint_as_float(b1 & 0xffff0000u));
+                } else {
+                    w[c] = Mma<T>::pack(p0, p1);
+                }
                 lp[c & 3] += p0 + p1;
             }
+            if (!settled) {
+                ok = wait_warp(&o_done[qtile], (j - 1) & 1, abort_flag);
+                if (!ok) break;
+                fence_after_sync();
+            }
             tmem_st32(tmem + lane_base + p_col, w);
-            tmem_st32(tmem + lane_base + p_col + kKeys / 2, r);
+            if (Fmt<T>::two_parts) tmem_st32(tmem + lane_base + p_col + kKeys / 2, r);
             l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
             tmem_wait_st();
             fence_before_sync();
