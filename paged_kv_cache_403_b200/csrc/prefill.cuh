@@ -20,10 +20,13 @@
 //   warp 8           tensor-core issue (one lane): S_t = Q_t K^T (M=128, N=64, both
 //                    operands in shared memory) and O_t += P_t V (M=128, N=head_dim,
 //                    per part of P; A = P from TMEM, B = V from shared memory);
-//   warp 9           TMA producer: 64-key tiles of K and V (2-D tensor loads, 128-byte
-//                    swizzle) into a 4-stage ring, walking the block table.
-// P never touches shared memory, which leaves room for four K/V stages: a tile is
-// requested four tiles before the tensor core needs it.
+//   warp 9           TMA producer: 128-key tiles of K and V (2-D tensor loads, 128-byte
+//                    swizzle) into a 2-stage ring, walking the block table.
+// Tiles of 128 keys make S = Q K^T an M=128, N=128 product: at N=64 the tensor core ran
+// it at about a third of its rate.  TMEM then holds O and S of both query tiles (512
+// columns), so P is written over S in place: the 16 columns of each 16-key group of S
+// take that group's P (8 columns of high parts, 8 of low parts), and the next S of the
+// tile is issued after the P V that reads them (one thread's tcgen05.mma run in order).
 // The two tiles ping-pong: while one warpgroup computes exponentials the tensor core
 // works on the other tile.  Every hand-off is an mbarrier; every wait is bounded and
 // sets a shared abort flag that all roles check; TMEM is always freed.  Key rows past
@@ -33,20 +36,20 @@ namespace prefill {
 
 constexpr int kRows = 128;           // MMA M: rows of one query tile
 constexpr int kTiles = 2;            // query tiles per CTA (ping-pong)
-constexpr int kKeys = 64;            // keys per K/V tile
+constexpr int kKeys = 128;           // keys per K/V tile
 constexpr int kSoftmaxThreads = kTiles * kRows;
 constexpr int kThreads = kSoftmaxThreads + 64;   // + tensor-core issue warp + TMA warp
 constexpr int kMmaWarp = kSoftmaxThreads / 32, kTmaWarp = kMmaWarp + 1;
 constexpr int kD = 128;              // head_dim
-// TMEM columns: O_A [0,128) O_B [128,256) S_A [256,320) S_B [320,384) P_A [384,448)
-// P_B [448,512); a P region holds the 64 keys' high halves in its first 32 columns
-// (two 16-bit values per column) and the low halves in the next 32.
+// TMEM columns: O_A [0,128) O_B [128,256) S_A [256,384) S_B [384,512); after the
+// softmax, columns [16g, 16g+8) of S_t hold the high parts of keys 16g..16g+15 of P_t
+// (two 16-bit values per column) and [16g+8, 16g+16) the low parts.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kOCol = 0, kSCol = 256, kPCol = 384;
+constexpr uint32_t kOCol = 0, kSCol = 256;
 constexpr int kQBytes = kRows * kD * 2;         // 32 KB per tile: [2 halves][128 rows][128 B]
-constexpr int kKVBytes = kKeys * kD * 2;        // 16 KB: [2 halves][64 rows][128 B]
-constexpr int kStages = 4;
-constexpr int kNumBars = 3 * kTiles + 2 * kStages;
+constexpr int kKVBytes = kKeys * kD * 2;        // 32 KB: [2 halves][128 rows][128 B]
+constexpr int kStages = 2;
+constexpr int kNumBars = 3 * kTiles + 4 * kStages;   // s_full, p_full, o_done; k/v full, empty
 constexpr int kSmemBytes = 1024 + kTiles * kQBytes + kStages * 2 * kKVBytes + kNumBars * 8 + 16;
 
 // --- tcgen05 wrappers --------------------------------------------------------------
@@ -196,8 +199,10 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
     unsigned char *sQ = smem;                                       // tile t at t * kQBytes
     unsigned char *sKV = sQ + kTiles * kQBytes;                     // stage st: K then V
     uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + kStages * 2 * kKVBytes);
-    uint64_t *kv_full = bars, *kv_empty = bars + kStages;
-    uint64_t *s_full = bars + 2 * kStages, *p_full = s_full + kTiles, *o_done = p_full + kTiles;
+    // K and V slots are released separately: a K tile is free once both query tiles'
+    // S used it, long before P V is done with the V tile beside it
+    uint64_t *k_full = bars, *k_empty = bars + kStages, *v_full = bars + 2 * kStages, *v_empty = bars + 3 * kStages;
+    uint64_t *s_full = bars + 4 * kStages, *p_full = s_full + kTiles, *o_done = p_full + kTiles;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -226,8 +231,10 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&kv_full[i], 1);
-            mbar_init(&kv_empty[i], 1);
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
         }
         for (int t = 0; t < kTiles; ++t) {
             mbar_init(&s_full[t], 1);
@@ -271,7 +278,6 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
         const int32_t *trow = p.tables + (size_t)s * p.max_blocks;
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j % kStages;
-            if (j >= kStages && !wait_warp(&kv_empty[st], ((j / kStages) - 1) & 1, abort_flag)) break;
             int blk = 0;
             if (lane < BLOCKS_PER_TILE) {
                 const int lb = j * BLOCKS_PER_TILE + lane;
@@ -281,28 +287,38 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                     blk = 0;
                 }
             }
-            if (lane == 0) mbar_arrive_expect_tx(&kv_full[st], 2 * kKVBytes);
+            unsigned char *k_dst = sKV + st * 2 * kKVBytes;
+            for (int kv = 0; kv < 2; ++kv) {
+                uint64_t *full = kv == 0 ? &k_full[st] : &v_full[st];
+                uint64_t *empty = kv == 0 ? &k_empty[st] : &v_empty[st];
+                if (j >= kStages && !wait_warp(empty, ((j / kStages) - 1) & 1, abort_flag)) break;
+                if (lane == 0) mbar_arrive_expect_tx(full, kKVBytes);
 #pragma unroll
-            for (int b = 0; b < BLOCKS_PER_TILE; ++b) {
-                const int bb = __shfl_sync(0xffffffffu, blk, b);
-                if (lane == 0) {
-                    const int r0 = ((p.layer * p.num_blocks + bb) * p.num_kv_heads + g) * B;
-                    unsigned char *k_dst = sKV + st * 2 * kKVBytes;
-                    for (int h = 0; h < 2; ++h) {
-                        tma_load_2d(k_dst + h * (kKVBytes / 2) + b * B * 128, &p.tmap_k, h * 64, r0, &kv_full[st]);
-                        tma_load_2d(k_dst + kKVBytes + h * (kKVBytes / 2) + b * B * 128, &p.tmap_v, h * 64, r0,
-                                    &kv_full[st]);
+                for (int b = 0; b < BLOCKS_PER_TILE; ++b) {
+                    const int bb = __shfl_sync(0xffffffffu, blk, b);
+                    if (lane == 0) {
+                        const int r0 = ((p.layer * p.num_blocks + bb) * p.num_kv_heads + g) * B;
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_2d(k_dst + kv * kKVBytes + h * (kKVBytes / 2) + b * B * 128,
+                                        kv == 0 ? &p.tmap_k : &p.tmap_v, h * 64, r0, full);
                     }
                 }
             }
+            if (*abort_flag) break;
             __syncwarp();
         }
     } else if (warp == kMmaWarp) {
         // ---------------- tensor-core issue
-        // wait for tile j's keys/values; zero value rows past the sequence end
-        auto ready = [&](int j) -> bool {
+        // wait for tile j's keys
+        auto ready_k = [&](int j) -> bool {
+            if (!wait_warp(&k_full[j % kStages], (j / kStages) & 1, abort_flag)) return false;
+            fence_after_sync();
+            return true;
+        };
+        // wait for tile j's values; zero value rows past the sequence end
+        auto ready_v = [&](int j) -> bool {
             const int st = j % kStages;
-            if (!wait_warp(&kv_full[st], (j / kStages) & 1, abort_flag)) return false;
+            if (!wait_warp(&v_full[st], (j / kStages) & 1, abort_flag)) return false;
             const int first_bad = L - j * kKeys;
             if (first_bad < kKeys) {
                 unsigned char *v_st = sKV + st * 2 * kKVBytes + kKVBytes;
@@ -343,34 +359,42 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
         };
         auto issue_pv = [&](int t, int j) {
             if (lane == 0) {
-                const uint32_t pcol = tmem + kPCol + t * kKeys;
+                const uint32_t pcol = tmem + kSCol + t * kKeys;
                 const uint64_t vb = v_desc + (uint64_t)(((j % kStages) * 2 * kKVBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < kKeys / 16; ++kk) {
                     const uint64_t b = vb + (uint64_t)((kk * 16 * 128) >> 4);
-                    umma_ts(tmem + kOCol + t * kD, pcol + kk * 8, b, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
-                    if (Fmt<T>::two_parts) umma_ts(tmem + kOCol + t * kD, pcol + kKeys / 2 + kk * 8, b, IDESC_O, 1u);
+                    umma_ts(tmem + kOCol + t * kD, pcol + kk * 16, b, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+                    if (Fmt<T>::two_parts) umma_ts(tmem + kOCol + t * kD, pcol + kk * 16 + 8, b, IDESC_O, 1u);
                 }
                 umma_commit(&o_done[t]);
             }
             __syncwarp();
         };
-        bool ok = ready(0);
-        if (ok)
+        bool ok = ready_k(0);
+        if (ok) {
             for (int t = 0; t < n_qt; ++t) issue_s(t, 0);
+            if (lane == 0) umma_commit(&k_empty[0]);   // K(0) free once both S(0) are done
+            __syncwarp();
+        }
         for (int j = 0; j < n_tiles && ok; ++j) {
             for (int t = 0; t < n_qt && ok; ++t) {
                 ok = wait_warp(&p_full[t], j & 1, abort_flag);   // softmax t read S_t(j), wrote P_t(j)
                 if (!ok) break;
                 fence_after_sync();
-                // next scores first: the softmax of S_t(j+1) then runs while P_t(j) V(j) does
+                // P_t(j) V(j) first: S_t(j+1) overwrites the columns P_t(j) is read from
+                if (t == 0) ok = ready_v(j);
+                if (!ok) break;
+                issue_pv(t, j);
                 if (j + 1 < n_tiles) {
-                    if (t == 0) ok = ready(j + 1);
+                    if (t == 0) ok = ready_k(j + 1);
                     if (ok) issue_s(t, j + 1);
                 }
-                if (ok) issue_pv(t, j);
             }
-            if (ok && lane == 0) umma_commit(&kv_empty[j % kStages]);
+            if (ok && lane == 0) {
+                umma_commit(&v_empty[j % kStages]);
+                if (j + 1 < n_tiles) umma_commit(&k_empty[(j + 1) % kStages]);
+            }
             __syncwarp();
         }
     } else {
@@ -379,7 +403,6 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
         const int kmax = row_valid ? P0 + my_t : -1;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t s_col = kSCol + qtile * kKeys, o_col = kOCol + qtile * kD;
-        const uint32_t p_col = kPCol + qtile * kKeys;
         const float sl = p.scale_log2;
         float m = -INFINITY, l = 0.f;
         bool ok = tile_used;
@@ -387,49 +410,42 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             ok = wait_warp(&s_full[qtile], j & 1, abort_flag);
             if (!ok) break;
             fence_after_sync();
-            uint32_t sv[64];
-            {
-                uint32_t a[32], b[32];
-                tmem_ld32(tmem + lane_base + s_col, a);
-                tmem_ld32(tmem + lane_base + s_col + 32, b);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    sv[c] = a[c];
-                    sv[32 + c] = b[c];
-                }
-            }
             const int key0 = j * kKeys;
             // interior tiles need no mask; the last ones mask by select (keys past this
             // row's position or past the sequence end get weight 0)
             const bool full_tile = key0 + kKeys - 1 <= kmax && key0 + kKeys <= L;
-            if (!full_tile) {
+            auto load_chunk = [&](int c, uint32_t (&v)[32]) {
+                tmem_ld32(tmem + lane_base + s_col + 32 * c, v);
+                tmem_wait_ld();
+                if (!full_tile) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (!(key0 + c <= kmax && key0 + c < L)) sv[c] = __float_as_uint(-INFINITY);
-            }
-            // maximum on raw scores (scale > 0 keeps the order), as a tree of 8 chains
+                    for (int e = 0; e < 32; ++e) {
+                        const int key = key0 + 32 * c + e;
+                        if (!(key <= kmax && key < L)) v[e] = __float_as_uint(-INFINITY);
+                    }
+                }
+            };
+            // pass 1: maximum on raw scores (scale > 0 keeps the order), 8 chains
             float mx8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sv[e]);
+            for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
 #pragma unroll
-            for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sv[c]));
+            for (int c = 0; c < kKeys / 32; ++c) {
+                uint32_t v[32];
+                load_chunk(c, v);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
+            }
             const float smax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                      fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             const float tmax = smax * sl;
-            // P_t(j-1) V(j-1) may still be running: O_t and the P_t region are only touched
-            // after it completes (the exponentials below do not need it).  The rescale
-            // decision is taken per warp (tcgen05.ld / st are warp-wide); rows that do
-            // not need it scale by 1.
+            // The rescale decision is taken per warp (tcgen05.ld / st are warp-wide); rows
+            // that do not need it scale by 1.  P_t(j-1) V(j-1) completed before S_t(j)
+            // (issued after it on the same thread), so O_t is settled.
             const bool need = tmax > m + kRescaleThreshold;
-            bool settled = j == 0;
             if (__any_sync(0xffffffffu, need)) {
                 const float f = need ? ex2(m - tmax) : 1.f;
                 if (j > 0) {
-                    ok = wait_warp(&o_done[qtile], (j - 1) & 1, abort_flag);
-                    if (!ok) break;
-                    fence_after_sync();
-                    settled = true;
 #pragma unroll
                     for (int c0 = 0; c0 < kD; c0 += 32) {
                         uint32_t o[32];
@@ -446,33 +462,35 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                     m = tmax;
                 }
             }
-            // p = 2^(s * scale_log2 - m): one FMA and one ex2 per score (-inf -> 0); the
-            // high and low 16-bit parts go back to this row's TMEM lane
+            // pass 2: p = 2^(s * scale_log2 - m), one FMA and one ex2 per score (-inf -> 0),
+            // written over the chunk's own S columns: per 16 keys, 8 columns of high parts
+            // then 8 of low parts
             const float neg_m = m == -INFINITY ? 0.f : -m;
             float lp[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t w[32], r[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float p0 = ex2(fmaf(__uint_as_float(sv[2 * c]), sl, neg_m));
-                const float p1 = ex2(fmaf(__uint_as_float(sv[2 * c + 1]), sl, neg_m));
-                if (Fmt<T>::two_parts) {
-                    // high halves of the two fp32 words = their bf16 truncations; the
-                    // remainders are exact in fp32 and rounded once to bf16
-                    const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-                    w[c] = byte_perm(b0, b1, 0x7632u);
-                    r[c] = Mma<T>::pack(p0 - __uint_as_float(b0 & 0xffff0000u), p1 - __uint_as_float(b1 & 0xffff0000u));
-                } else {
-                    w[c] = Mma<T>::pack(p0, p1);
+            for (int c = 0; c < kKeys / 32; ++c) {
+                uint32_t v[32], pw[32];
+                load_chunk(c, v);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = ex2(fmaf(__uint_as_float(v[2 * e]), sl, neg_m));
+                    const float p1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), sl, neg_m));
+                    const int slot = (e >> 3) * 16 + (e & 7);     // key group e/8, pair e%8
+                    if (Fmt<T>::two_parts) {
+                        // high halves of the two fp32 words = their bf16 truncations; the
+                        // remainders are exact in fp32 and rounded once to bf16
+                        const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+                        pw[slot] = byte_perm(b0, b1, 0x7632u);
+                        pw[slot + 8] = Mma<T>::pack(p0 - __uint_as_float(b0 & 0xffff0000u),
+                                                    p1 - __uint_as_float(b1 & 0xffff0000u));
+                    } else {
+                        pw[slot] = Mma<T>::pack(p0, p1);
+                        pw[slot + 8] = 0u;
+                    }
+                    lp[e & 3] += p0 + p1;
                 }
-                lp[c & 3] += p0 + p1;
+                tmem_st32(tmem + lane_base + s_col + 32 * c, pw);
             }
-            if (!settled) {
-                ok = wait_warp(&o_done[qtile], (j - 1) & 1, abort_flag);
-                if (!ok) break;
-                fence_after_sync();
-            }
-            tmem_st32(tmem + lane_base + p_col, w);
-            if (Fmt<T>::two_parts) tmem_st32(tmem + lane_base + p_col + kKeys / 2, r);
             l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
             tmem_wait_st();
             fence_before_sync();
