@@ -155,9 +155,9 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volati
 
 // Operand format code of the instruction descriptor, and how P enters P V: bf16 P
 // keeps 8 significant bits, too few for the 2e-3 bound on peaky rows, so a bf16 P is a
-// high part (the truncation of p to bf16, taken with one byte permute) plus the bf16
-// rounding of the exact remainder (~16 bits together, two products); an fp16 P keeps 11
-// bits and enters once.
+// high part (the truncation of p to bf16) plus the truncation of the exact remainder
+// p - high (>= 14 bits together, two products), both taken with byte permutes so the
+// conversion unit only computes exponentials; an fp16 P keeps 11 bits and enters once.
 template <typename T>
 struct Fmt;
 template <>
@@ -176,6 +176,7 @@ __device__ __forceinline__ uint32_t byte_perm(uint32_t a, uint32_t b, uint32_t s
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
     return r;
 }
+
 
 struct Params {
     CUtensorMap tmap_k;
@@ -473,16 +474,17 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                 load_chunk(c, v);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(__uint_as_float(v[2 * e]), sl, neg_m));
-                    const float p1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), sl, neg_m));
+                    const float x0 = fmaf(__uint_as_float(v[2 * e]), sl, neg_m);
+                    const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), sl, neg_m);
+                    const float p0 = ex2(x0), p1 = ex2(x1);
                     const int slot = (e >> 3) * 16 + (e & 7);     // key group e/8, pair e%8
                     if (Fmt<T>::two_parts) {
                         // high halves of the two fp32 words = their bf16 truncations; the
-                        // remainders are exact in fp32 and rounded once to bf16
+                        // remainders (exact in fp32, >= 0) truncated the same way
                         const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
                         pw[slot] = byte_perm(b0, b1, 0x7632u);
-                        pw[slot + 8] = Mma<T>::pack(p0 - __uint_as_float(b0 & 0xffff0000u),
-                                                    p1 - __uint_as_float(b1 & 0xffff0000u));
+                        pw[slot + 8] = byte_perm(__float_as_uint(p0 - __uint_as_float(b0 & 0xffff0000u)),
+                                                 __float_as_uint(p1 - __uint_as_float(b1 & 0xffff0000u)), 0x7632u);
                     } else {
                         pw[slot] = Mma<T>::pack(p0, p1);
                         pw[slot + 8] = 0u;
