@@ -11,8 +11,11 @@
 // One CTA per (256 query rows, KV head, sequence): two 128-row tiles A and B whose rows
 // are (token, query head of the GQA group) pairs, row = token * G + head, so every
 // query head of the group shares each key/value tile.  Warp roles:
-//   warps 0-3 / 4-7  softmax of tile A / B: thread = row = TMEM lane; tcgen05.ld of the
-//                    row's 64 scores, causal / length mask by select, base-2 online
+//   warps 0-15       softmax: warp w serves tile (w / 4) % 2, rows 32 (w % 4) .. +31 (its
+//                    TMEM lane quarter) and keys / O columns 64 (w / 8) .. +63, so two
+//                    threads share a row and exchange their partial maxima (and at the
+//                    end their sums) through shared memory; per row: tcgen05.ld of the
+//                    scores, causal / length mask by select, base-2 online
 //                    softmax with a lazily moved maximum (the O row is rescaled in TMEM
 //                    only when a score passes the running maximum by 2^8), P written
 //                    back to TMEM (tcgen05.st) as the A operand of P V: for bf16 a
@@ -37,9 +40,10 @@ namespace prefill {
 constexpr int kRows = 128;           // MMA M: rows of one query tile
 constexpr int kTiles = 2;            // query tiles per CTA (ping-pong)
 constexpr int kKeys = 128;           // keys per K/V tile
-constexpr int kSoftmaxThreads = kTiles * kRows;
-constexpr int kThreads = kSoftmaxThreads + 64;   // + tensor-core issue warp + TMA warp
-constexpr int kMmaWarp = kSoftmaxThreads / 32, kTmaWarp = kMmaWarp + 1;
+constexpr int kHalves = 2;           // softmax threads per row (each: 64 keys, 64 O columns)
+constexpr int kSoftmaxWarps = kTiles * kRows * kHalves / 32;
+constexpr int kThreads = kSoftmaxWarps * 32 + 64;   // + tensor-core issue warp + TMA warp
+constexpr int kMmaWarp = kSoftmaxWarps, kTmaWarp = kMmaWarp + 1;
 constexpr int kD = 128;              // head_dim
 // TMEM columns: O_A [0,128) O_B [128,256) S_A [256,384) S_B [384,512); after the
 // softmax, columns [16g, 16g+8) of S_t hold the high parts of keys 16g..16g+15 of P_t
@@ -49,8 +53,11 @@ constexpr uint32_t kOCol = 0, kSCol = 256;
 constexpr int kQBytes = kRows * kD * 2;         // 32 KB per tile: [2 halves][128 rows][128 B]
 constexpr int kKVBytes = kKeys * kD * 2;        // 32 KB: [2 halves][128 rows][128 B]
 constexpr int kStages = 2;
-constexpr int kNumBars = 3 * kTiles + 4 * kStages;   // s_full, p_full, o_done; k/v full, empty
-constexpr int kSmemBytes = 1024 + kTiles * kQBytes + kStages * 2 * kKVBytes + kNumBars * 8 + 16;
+// s_full, p_full, o_done per tile; k/v full, empty per stage; one row-exchange barrier
+// per (tile, lane quarter)
+constexpr int kNumBars = 3 * kTiles + 4 * kStages + kTiles * 4;
+constexpr int kXchBytes = 2 * kTiles * kHalves * kRows * 4;   // [parity][tile][half][row] floats
+constexpr int kSmemBytes = 1024 + kTiles * kQBytes + kStages * 2 * kKVBytes + kNumBars * 8 + 16 + kXchBytes;
 
 // --- tcgen05 wrappers --------------------------------------------------------------
 // Shared-memory matrix descriptor, 128-byte swizzle: start address, leading and stride
@@ -204,8 +211,10 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
     // S used it, long before P V is done with the V tile beside it
     uint64_t *k_full = bars, *k_empty = bars + kStages, *v_full = bars + 2 * kStages, *v_empty = bars + 3 * kStages;
     uint64_t *s_full = bars + 4 * kStages, *p_full = s_full + kTiles, *o_done = p_full + kTiles;
+    uint64_t *x_bar = o_done + kTiles;                               // [tile][quarter]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float *xch = reinterpret_cast<float *>(tmem_slot + 4);           // 16-byte aligned
 
     const int s = blockIdx.z;
     const int g = blockIdx.y;
@@ -239,8 +248,9 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
         }
         for (int t = 0; t < kTiles; ++t) {
             mbar_init(&s_full[t], 1);
-            mbar_init(&p_full[t], 4);        // the four warps of the tile's softmax group
+            mbar_init(&p_full[t], 4 * kHalves);   // the eight warps of the tile's softmax group
             mbar_init(&o_done[t], 1);
+            for (int qq = 0; qq < 4; ++qq) mbar_init(&x_bar[t * 4 + qq], kHalves);
         }
         *abort_flag = 0;
         mbar_fence_init();
@@ -251,13 +261,16 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // query rows: tile t = tid / 128, row r = tid % 128; rows past the chunk are zero
-    const int qtile = tid / kRows;
-    const int row = tid % kRows;
+    // softmax warp w: tile (w / 4) % 2, lane quarter w % 4, key / column half w / 8; the
+    // half-0 warps load the query rows (rows past the chunk are zero)
+    const int quarter = warp & 3;
+    const int qtile = (warp >> 2) & 1;
+    const int half = warp >> 3;
+    const int row = quarter * 32 + lane;
     const int my_t = t0 + (qtile * kRows + row) / group;
     const int my_h = g * group + row % group;
-    const bool row_valid = tid < kSoftmaxThreads && my_t < C;
-    if (tid < kSoftmaxThreads) {
+    const bool row_valid = warp < kSoftmaxWarps && my_t < C;
+    if (warp < kSoftmaxWarps && half == 0) {
         const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.q) +
                                                             ((size_t)(q0 + (row_valid ? my_t : 0)) * p.num_q_heads + my_h) * kD);
         unsigned char *dst = sQ + qtile * kQBytes;
@@ -399,11 +412,23 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             __syncwarp();
         }
     } else {
-        // ---------------- softmax of tile qtile, row = TMEM lane
+        // ---------------- softmax of tile qtile, row = TMEM lane, keys / O columns of `half`
         const bool tile_used = qtile < n_qt;
         const int kmax = row_valid ? P0 + my_t : -1;
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t s_col = kSCol + qtile * kKeys, o_col = kOCol + qtile * kD;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t s_col = kSCol + qtile * kKeys + half * (kKeys / kHalves);
+        const uint32_t o_col = kOCol + qtile * kD + half * (kD / kHalves);
+        uint64_t *xb = &x_bar[qtile * 4 + quarter];
+        // the partner thread (same row, other half) meets here; a bounded wait
+        auto exchange = [&](int phase, float mine, float &theirs) -> bool {
+            float *x = xch + ((phase & 1) * kTiles + qtile) * kHalves * kRows;
+            x[half * kRows + row] = mine;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xb);
+            if (!wait_warp(xb, phase & 1, abort_flag)) return false;
+            theirs = x[(1 - half) * kRows + row];
+            return true;
+        };
         const float sl = p.scale_log2;
         float m = -INFINITY, l = 0.f;
         bool ok = tile_used;
@@ -411,10 +436,11 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             ok = wait_warp(&s_full[qtile], j & 1, abort_flag);
             if (!ok) break;
             fence_after_sync();
-            const int key0 = j * kKeys;
+            const int key0 = j * kKeys + half * (kKeys / kHalves);
+            constexpr int kMine = kKeys / kHalves;
             // interior tiles need no mask; the last ones mask by select (keys past this
             // row's position or past the sequence end get weight 0)
-            const bool full_tile = key0 + kKeys - 1 <= kmax && key0 + kKeys <= L;
+            const bool full_tile = key0 + kMine - 1 <= kmax && key0 + kMine <= L;
             auto load_chunk = [&](int c, uint32_t (&v)[32]) {
                 tmem_ld32(tmem + lane_base + s_col + 32 * c, v);
                 tmem_wait_ld();
@@ -431,15 +457,18 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
 #pragma unroll
             for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < kKeys / 32; ++c) {
+            for (int c = 0; c < kMine / 32; ++c) {
                 uint32_t v[32];
                 load_chunk(c, v);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
             }
-            const float smax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+            const float pmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                      fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-            const float tmax = smax * sl;
+            float other;
+            ok = exchange(j, pmax, other);
+            if (!ok) break;
+            const float tmax = fmaxf(pmax, other) * sl;     // both halves of the row agree
             // The rescale decision is taken per warp (tcgen05.ld / st are warp-wide); rows
             // that do not need it scale by 1.  P_t(j-1) V(j-1) completed before S_t(j)
             // (issued after it on the same thread), so O_t is settled.
@@ -448,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                 const float f = need ? ex2(m - tmax) : 1.f;
                 if (j > 0) {
 #pragma unroll
-                    for (int c0 = 0; c0 < kD; c0 += 32) {
+                    for (int c0 = 0; c0 < kD / kHalves; c0 += 32) {
                         uint32_t o[32];
                         tmem_ld32(tmem + lane_base + o_col + c0, o);
                         tmem_wait_ld();
@@ -469,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             const float neg_m = m == -INFINITY ? 0.f : -m;
             float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < kKeys / 32; ++c) {
+            for (int c = 0; c < kMine / 32; ++c) {
                 uint32_t v[32], pw[32];
                 load_chunk(c, v);
 #pragma unroll
@@ -500,12 +529,15 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             if (lane == 0) mbar_arrive(&p_full[qtile]);
         }
         if (ok) ok = wait_warp(&o_done[qtile], (n_tiles - 1) & 1, abort_flag);
+        float l_other = 0.f;
+        if (ok) ok = exchange(n_tiles, l, l_other);       // the row's sum over both halves
         if (ok) {
             fence_after_sync();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            const size_t orow = ((size_t)(q0 + my_t) * p.num_q_heads + my_h) * kD;
+            const float lt = l + l_other;
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            const size_t orow = ((size_t)(q0 + my_t) * p.num_q_heads + my_h) * kD + half * (kD / kHalves);
 #pragma unroll
-            for (int c0 = 0; c0 < kD; c0 += 32) {
+            for (int c0 = 0; c0 < kD / kHalves; c0 += 32) {
                 uint32_t o[32];
                 tmem_ld32(tmem + lane_base + o_col + c0, o);
                 tmem_wait_ld();
