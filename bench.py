@@ -57,6 +57,8 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seqs", type=int, default=24)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for the CPU baseline")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"],
+                    help="prefill workload: cache / query type (bf16 P enters P.V as two products, fp16 P once)")
     ap.add_argument("--kv-dtype", default="native", choices=["native", "fp8"],
                     help="native: the workload's 16-bit cache; fp8: E4M3 codes + per-row scale bytes "
                          "(queries and appended rows keep the workload's type)")
@@ -771,10 +773,11 @@ def run_prefill(args):
     import paged_kv_cache_403_b200 as pa
     from synthetic import workloads as wl
     torch.cuda.set_device(0)
-    r = wl.chunked_prefill()
+    r = wl.chunked_prefill(dtype=args.dtype)
     sh = r["shape"]
     c = prefill_setup(torch, r)
-    out = torch.empty((c["rows"], sh.num_q_heads, sh.head_dim), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((c["rows"], sh.num_q_heads, sh.head_dim),
+                      dtype=torch.bfloat16 if args.dtype == "bf16" else torch.float16, device="cuda")
     st = torch.cuda.current_stream()
     scale = 1.0 / math.sqrt(sh.head_dim)
 
@@ -811,9 +814,9 @@ def run_prefill(args):
     line = {"metric": "paged chunked-prefill attention TFLOP/s and prefill tokens/s", "impl": "ours",
             "value": round(c["flops"] * args.steps / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
-            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "higher_is_better": True, "dtype": args.dtype, "data": "synthetic",
             "config": {"workload": "chunked_prefill: 32 seqs, lengths U[1024,4096], last 512 tokens as queries, "
-                                   "block 16, 32 q / 8 KV heads, d128, bf16"},
+                                   "block 16, 32 q / 8 KV heads, d128, " + args.dtype},
             "prefill_tokens_per_s": round(c["rows"] * args.steps / (ms * 1e-3), 1),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "traffic": None, "kernel": "paged_prefill_kernel",

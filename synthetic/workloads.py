@@ -146,14 +146,15 @@ def system_block_keys(n_blocks: int, system_uid: int = SYSTEM_UID):
     return [(system_uid << 32) | i for i in range(n_blocks)]
 
 
-def chunked_prefill(seed: int = 7, n: int = 32, lo: int = 1024, hi: int = 4096, chunk: int = 512) -> dict:
+def chunked_prefill(seed: int = 7, n: int = 32, lo: int = 1024, hi: int = 4096, chunk: int = 512,
+                    dtype: str = "bf16") -> dict:
     """Chunked prefill: n sequences with total lengths U[lo, hi]; the last `chunk` tokens
     of each are the queries (their keys and values are already cached).  Block 16,
-    32 q / 8 KV heads, d128, bf16, 1 layer."""
+    32 q / 8 KV heads, d128, bf16 (or fp16), 1 layer."""
     rng = np.random.default_rng(seed)
     lens = rng.integers(lo, hi + 1, size=n)
     chunks = np.minimum(lens, chunk)
-    shape = Shape(1, 16, 32, 8, 128, "bf16", int(sum(-(-int(L) // 16) for L in lens)) + 16,
+    shape = Shape(1, 16, 32, 8, 128, dtype, int(sum(-(-int(L) // 16) for L in lens)) + 16,
                   kv_scale=1.0 / math.sqrt(128.0))
     order = rng.permutation(shape.num_blocks).astype(np.int32)
     return dict(name="chunked_prefill", seed=seed, shape=shape, lens=lens, chunks=chunks, order=order)
