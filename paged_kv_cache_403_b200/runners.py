@@ -80,7 +80,7 @@ def decode_step(cache: PagedCache, gen: DeviceGen, sids, uids, num_q_heads, max_
     slots_dev = torch.from_numpy(np.ascontiguousarray(slots)).to(dev)
     tables_dev = torch.from_numpy(tables).to(dev)
     lens_dev = torch.from_numpy(lens).to(dev)
-    out_dtype = out_dtype or TORCH_DTYPES[cache.dtype]
+    out_dtype = out_dtype or TORCH_DTYPES[cache.act_dtype]
     if workspace is None:
         workspace = cache.workspace(len(sids), num_q_heads, max_blocks, split_tokens)
     rec = StepRecord(list(sids), list(uids), positions, slots.copy(), cow.copy(), tables.copy(), lens.copy())
@@ -96,10 +96,19 @@ def decode_step(cache: PagedCache, gen: DeviceGen, sids, uids, num_q_heads, max_
     return rec
 
 
-def run_static(recipe, split_tokens=0, out_dtype=None, keep_layers=None, device="cuda"):
+def make_cache(shape, order, device="cuda", kv_fp8=False):
+    """The workload's cache: its own 16-bit type, or an FP8 cache whose queries and
+    appended rows keep that type."""
+    if kv_fp8:
+        return PagedCache(shape.num_layers, shape.num_blocks, shape.block_size, shape.num_kv_heads, shape.head_dim,
+                          "fp8", order, device, act_dtype=shape.dtype)
+    return PagedCache.from_shape(shape, order, device)
+
+
+def run_static(recipe, split_tokens=0, out_dtype=None, keep_layers=None, device="cuda", kv_fp8=False):
     """tiny / worked_example / large_pool: prefill every sequence, then one decode step."""
     shape = recipe["shape"]
-    cache = PagedCache.from_shape(shape, recipe["order"], device)
+    cache = make_cache(shape, recipe["order"], device, kv_fp8)
     gen = DeviceGen(recipe["seed"], shape, device)
     lens = [int(L) for L in recipe["lens"]]
     sids = [cache.add() for _ in lens]
@@ -147,11 +156,11 @@ class ContinuousBatch:
     """Continuous-batch workload: fixed batch slots, stops drawn per step, replacements
     admitted (prefilled) at the start of the next step."""
 
-    def __init__(self, recipe, device="cuda", max_blocks=None):
+    def __init__(self, recipe, device="cuda", max_blocks=None, kv_fp8=False):
         self.recipe = recipe
         self.shape = shape = recipe["shape"]
         self.sched = recipe["schedule"]
-        self.cache = PagedCache.from_shape(shape, recipe["order"], device)
+        self.cache = make_cache(shape, recipe["order"], device, kv_fp8)
         self.gen = DeviceGen(recipe["seed"], shape, device)
         self.device = device
         n = len(self.sched.initial)

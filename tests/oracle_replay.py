@@ -102,3 +102,23 @@ def sequence_attention(shape, seed, layer, uid, length, q_uid, q_pos, writer=Non
     q = sv.rows(sv.KIND_Q, seed, layer, [q_uid], [q_pos], shape.num_q_heads, d, shape.q_scale, shape.dtype)
     return oracle.paged_decode(kp, vp, shape.dtype, np.arange(nblk, dtype=np.int32)[None], np.array([length]),
                                q, 1.0 / math.sqrt(d))[0]
+
+
+def sequence_attention_fp8(shape, seed, layer, uid, length, q_uid, q_pos):
+    """As sequence_attention, over an FP8 cache: the regenerated rows (in the workload's
+    type) are quantised by the oracle's own quantiser, then attended in fp64."""
+    from oracle.fp8 import quantize_rows
+    B, hkv, d = shape.block_size, shape.num_kv_heads, shape.head_dim
+    pos = np.arange(length)
+    wu = np.full(length, uid)
+    kc, ks = quantize_rows(oracle.widen(sv.rows(sv.KIND_K, seed, layer, wu, pos, hkv, d, shape.kv_scale, shape.dtype),
+                                        shape.dtype).astype(np.float32))
+    vc, vs = quantize_rows(oracle.widen(sv.rows(sv.KIND_V, seed, layer, wu, pos, hkv, d, shape.kv_scale, shape.dtype),
+                                        shape.dtype).astype(np.float32))
+    nblk = -(-length // B)
+    pad = nblk * B - length
+    lay = lambda a: np.ascontiguousarray(np.concatenate([a, np.zeros((pad,) + a.shape[1:], a.dtype)])  # noqa: E731
+                                         .reshape((nblk, B) + a.shape[1:]).swapaxes(1, 2))
+    q = sv.rows(sv.KIND_Q, seed, layer, [q_uid], [q_pos], shape.num_q_heads, d, shape.q_scale, shape.dtype)
+    return oracle.paged_decode_fp8(lay(kc), lay(vc), lay(ks), lay(vs), np.arange(nblk, dtype=np.int32)[None],
+                                   np.array([length]), q, shape.dtype, 1.0 / math.sqrt(d))[0]

@@ -322,3 +322,59 @@ def test_fp8_pool_rejections():
         pa.pa_pool_create(1, 4, 16, 2, D, "fp8", act_dtype="f32")
     assert e.value.status == pa.PA_ERR_INVALID_ARG
     assert pa.pa_launch_count() == before
+
+
+# ------------------------------------------------------------------ full sizes
+@pytest.mark.slow
+def test_continuous_batch_fp8_full_size_sampled():
+    """256 sequences, 64 steps, FP8 cache, bf16 output, split 2048 as the benchmark times
+    them; sampled sequences against the oracle over their regenerated, oracle-quantised
+    histories, and sampled cache rows bit-exact against the oracle's quantiser."""
+    from oracle_replay import sequence_attention_fp8
+    from paged_kv_cache_403_b200.runners import ContinuousBatch
+    from synthetic import workloads as wl
+    r = wl.continuous_batch()
+    sh = r["shape"]
+    cb = ContinuousBatch(r, kv_fp8=True)
+    rng = np.random.default_rng(0)
+    for t in range(64):
+        rec = cb.step(split_tokens=2048)
+        if t in (0, 33, 63):
+            lens = rec.lens
+            picks = set(rng.choice(len(lens), size=5, replace=False).tolist())
+            picks |= {int(np.argmax(lens)), int(np.argmin(lens))}
+            out = rec.outputs[0].detach().cpu().to(torch.float64).numpy()
+            for i in sorted(picks):
+                ref = sequence_attention_fp8(sh, r["seed"], 0, rec.uids[i], int(lens[i]), rec.uids[i],
+                                             int(rec.positions[i]))
+                check_close(out[i], ref, "bf16", "bf16", f"step {t} seq {i}")
+    kp, sc = host(cb.cache.k_pool), host(cb.cache.scales)
+    for i in range(0, 256, 37):
+        L = int(rec.lens[i])
+        blk, off = int(rec.tables[i][(L - 1) // 16]), (L - 1) % 16
+        row = sv.rows(sv.KIND_K, r["seed"], 0, [rec.uids[i]], [L - 1], 8, 128, sh.kv_scale, "bf16")
+        codes, scales = quantize(row, "bf16")
+        assert np.array_equal(kp[0, blk, :, off], codes[0]) and np.array_equal(sc[0, blk, :, 0, off], scales[0])
+
+
+@pytest.mark.slow
+def test_large_pool_fp8_sampled():
+    """384 sequences, lognormal lengths, 32 layers, block 32, FP8 cache (~50 GB), split 2048
+    as the benchmark times it; layers 0 and 31 sampled against the oracle."""
+    from oracle_replay import sequence_attention_fp8
+    from paged_kv_cache_403_b200.runners import run_static
+    from synthetic import workloads as wl
+    r = wl.large_pool(block_size=32)
+    sh = r["shape"]
+    cache, _, rec = run_static(r, split_tokens=2048, keep_layers={0, 31}, kv_fp8=True)
+    lens = rec.lens
+    picks = [int(np.argmax(lens)), int(np.argmin(lens)), int(np.argsort(lens)[len(lens) // 2])]
+    picks += [int(i) for i in np.nonzero(lens > 4096)[0][:2]]
+    for layer in (0, 31):
+        out = rec.outputs[layer].detach().cpu().to(torch.float64).numpy()
+        for i in picks:
+            ref = sequence_attention_fp8(sh, r["seed"], layer, rec.uids[i], int(lens[i]), rec.uids[i],
+                                         int(rec.positions[i]))
+            check_close(out[i], ref, "f16", "f16", f"layer {layer} seq {i}")
+    del cache
+    torch.cuda.empty_cache()
