@@ -57,3 +57,46 @@ def test_device_calls_without_device_memory_fail_cleanly():
         pa._check(pa._lib().pa_decode_attention(pool, 0, None, None, 0, None, 1, None, 1, 2, 1.0, 0,
                                                 None, 0, None))
     pa.pa_pool_destroy(pool)
+
+
+def test_fp8_pool_configuration_rules():
+    """FP8 pools: a 16-bit activation type is required, block sizes are multiples of 16,
+    the scale array attaches to FP8 pools only, and host bookkeeping works without device
+    memory; the swap record of a block carries its codes and its scale bytes."""
+    with pytest.raises(pa.PaError) as e:                    # no activation type given
+        pa.pa_pool_create(1, 8, 16, 2, 128, "fp8")
+    assert e.value.status == pa.PA_ERR_INVALID_ARG
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_pool_create(1, 8, 16, 2, 128, "fp8", act_dtype="f32")
+    assert e.value.status == pa.PA_ERR_INVALID_ARG
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_pool_create(1, 8, 8, 2, 128, "fp8", act_dtype="bf16")
+    assert e.value.status == pa.PA_ERR_UNSUPPORTED
+    bf = pa.pa_pool_create(1, 8, 16, 2, 128, "bf16")
+    with pytest.raises(pa.PaError) as e:                    # scales on a 16-bit pool
+        pa._check(pa._lib().pa_pool_set_scales(bf, 16))
+    assert e.value.status == pa.PA_ERR_INVALID_ARG
+    pa.pa_pool_destroy(bf)
+    p = pa.pa_pool_create(3, 40, 16, 2, 128, "fp8", act_dtype="bf16")
+    with pytest.raises(pa.PaError) as e:                    # misaligned scale array
+        pa._check(pa._lib().pa_pool_set_scales(p, 8))
+    assert e.value.status == pa.PA_ERR_INVALID_ARG
+    s = pa.pa_seq_add(p)
+    pa.pa_reserve_slots(p, [s], [50])                       # 4 blocks
+    # per block and layer: K and V codes (2 * 2 heads * 16 * 128) + scale bytes (2 heads * 2 * 16)
+    assert pa.pa_swap_bytes(p, s) == 4 * 3 * (2 * 2 * 16 * 128 + 2 * 2 * 16)
+    pa.pa_swap_out(p, s)                                    # bookkeeping only (no device pools)
+    pa.pa_swap_in(p, s)
+    assert pa.pa_seq_info(p, s)[0] == 50
+    pa.pa_pool_destroy(p)
+
+
+def test_decode_workspace_sizes_cover_every_part():
+    # n * max_splits range ids; with splits also partials (acc + (m, l)) and one counter
+    # per (sequence, query head); each part rounded up to 16 bytes
+    for n, hq, d, ms in [(1, 1, 64, 1), (7, 8, 128, 1), (7, 8, 128, 5), (256, 32, 128, 3)]:
+        parts = n * ms * hq
+        partials = -(-(parts * d * 4 + parts * 8) // 16) * 16 if ms > 1 else 0
+        order = -(-(n * ms * 4) // 16) * 16
+        counters = -(-(n * hq * 4) // 16) * 16 if ms > 1 else 0
+        assert pa.pa_decode_workspace_bytes(n, hq, d, ms) == partials + order + counters
