@@ -29,7 +29,10 @@ def clean_device_error():
     assert pa.pa_device_error(clear=True) == 0
 
 
-def prefill_case(lens, chunks, B=16, hq=8, hkv=2, dtype="bf16", kv_scale=None, seed=0, fill=None):
+def prefill_case(lens, chunks, B=16, hq=8, hkv=2, dtype="bf16", kv_scale=None, seed=0, fill=None, k_rows=None,
+                 q_rows=None):
+    """k_rows(total, rng) / q_rows(total, rng): optional fp32 replacements for the random
+    keys / queries (the oracle gets the same host rows)."""
     d = 128
     kv_scale = 1 / math.sqrt(d) if kv_scale is None else kv_scale
     rng = np.random.default_rng(seed)
@@ -43,11 +46,15 @@ def prefill_case(lens, chunks, B=16, hq=8, hkv=2, dtype="bf16", kv_scale=None, s
     slots, _ = cache.reserve(sids, lens)
     k = sv.narrow((rng.standard_normal((sum(lens), hkv, d)) * kv_scale).astype(np.float32), dtype)
     v = sv.narrow((rng.standard_normal((sum(lens), hkv, d)) * kv_scale).astype(np.float32), dtype)
+    if k_rows is not None:
+        k = sv.narrow(k_rows(sum(lens), rng).astype(np.float32), dtype)
     cache.append(0, dev(k, dtype), dev(v, dtype), torch.from_numpy(np.ascontiguousarray(slots)).cuda())
     max_blocks = max(-(-L // B) for L in lens)
     tables, ln = cache.tables(sids, max_blocks)
     q_start = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
     q = sv.narrow(rng.standard_normal((int(q_start[-1]), hq, d)).astype(np.float32), dtype)
+    if q_rows is not None:
+        q = sv.narrow(q_rows(int(q_start[-1]), rng).astype(np.float32), dtype)
     # oracle's own pool (host): the same rows placed by the oracle's block-manager replay
     from oracle.block_manager import BlockManagerModel
     from oracle.cache_model import append_rows, empty_pools
@@ -58,9 +65,9 @@ def prefill_case(lens, chunks, B=16, hq=8, hkv=2, dtype="bf16", kv_scale=None, s
     append_rows(kp, vp, 0, oslots, k, v)
     otables, olens = bm.dense_tables(osids, max_blocks)
     assert np.array_equal(np.array(otables), tables)
-    ref = oracle.paged_prefill(kp[0], vp[0], dtype, np.array(otables, np.int32), np.array(olens, np.int32),
-                               q_start, q, 1 / math.sqrt(d))
-    return dict(cache=cache, tables=torch.from_numpy(tables).cuda(), lens=torch.from_numpy(ln).cuda(),
+    oracle_args = (kp[0], vp[0], dtype, np.array(otables, np.int32), np.array(olens, np.int32), q_start)
+    ref = oracle.paged_prefill(*oracle_args, q, 1 / math.sqrt(d))
+    return dict(oracle_args=oracle_args, cache=cache, tables=torch.from_numpy(tables).cuda(), lens=torch.from_numpy(ln).cuda(),
                 q_start=torch.from_numpy(q_start).cuda(), q=dev(q, dtype), ref=ref, max_q=int(max(chunks)),
                 hq=hq, d=d, dtype=dtype, q_np=q, tables_np=tables, lens_np=ln)
 
@@ -120,6 +127,48 @@ def test_prefill_rejects_unsupported_shapes():
                                 torch.ones(1, dtype=torch.int32, device="cuda"),
                                 torch.tensor([0, 4], dtype=torch.int32, device="cuda"), 4, 0.1)
     assert e.value.status == pa.PA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("B", [16, 32])
+def test_prefill_key_tile_and_cta_boundaries(B):
+    """Keys around the 128-key tile edges and query chunks around the 64-token CTA span
+    (256 rows / GQA 4), including a chunk that starts exactly on a tile edge."""
+    lens = [127, 128, 129, 255, 256, 257, 384, 1024]
+    chunks = [63, 64, 65, 127, 128, 1, 256, 200]
+    c = prefill_case(lens, chunks, B=B, seed=6)
+    check_close(run(c), c["ref"], "f32", "bf16", f"boundaries B{B}")
+
+
+def test_prefill_empty_chunks_in_the_batch():
+    """Sequences without queries this pass (chunk 0) sit between ones with queries."""
+    c = prefill_case([50, 300, 40, 129], [0, 77, 0, 129], seed=7)
+    check_close(run(c), c["ref"], "f32", "bf16", "empty chunks")
+
+
+def test_prefill_rising_scores_and_large_queries():
+    """Keys whose scores keep rising along each sequence move the running maximum on
+    almost every tile (the warp-wide rescale of O in TMEM, agreed by both threads of a
+    row); a second case uses large query norms (very peaky rows)."""
+    d = 128
+    qdir = np.random.default_rng(8).standard_normal(d)
+    qdir /= np.linalg.norm(qdir)
+    lens = [900, 1500]
+
+    def ramp_keys(total, rng):
+        pos = np.concatenate([np.arange(L) / L for L in lens])
+        return ((-20 + 60 * pos)[:, None, None] * qdir[None, None, :] / 3 + rng.standard_normal((total, 2, d)) * 0.05)
+
+    c = prefill_case(lens, [300, 129], seed=9, k_rows=ramp_keys,
+                     q_rows=lambda total, rng: np.tile(qdir * 12, (total, 8, 1)))
+    check_close(run(c), c["ref"], "f32", "bf16", "rising scores")
+    c2 = prefill_case([600, 257], [257, 257], seed=10, q_rows=lambda total, rng: rng.standard_normal((total, 8, d)) * 12)
+    check_close(run(c2), c2["ref"], "f32", "bf16", "large queries")
+
+
+def test_prefill_long_sequence():
+    """An 8,704-token sequence: 68 key tiles for the last chunk's queries."""
+    c = prefill_case([8704, 600], [512, 96], seed=12)
+    check_close(run(c), c["ref"], "f32", "bf16", "long sequence")
 
 
 @pytest.mark.slow
