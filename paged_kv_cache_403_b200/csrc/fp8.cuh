@@ -211,10 +211,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
         L = p.max_blocks * B;
     }
     const int nblk = (L + B - 1) / B;
-    const int b0 = split * p.split_blocks;
-    if (b0 >= nblk) return;
-    const int ntiles = min(nblk, b0 + p.split_blocks) - b0;
-    const int nsplit = (nblk + p.split_blocks - 1) / p.split_blocks;
+    const SplitRange rg = split_range(nblk, p.split_blocks, split);
+    if (split >= rg.n) return;
+    const int b0 = rg.b0;
+    const int ntiles = rg.b1 - rg.b0;
+    const int nsplit = rg.n;
 
     unsigned char *scl = smem + SH::kRingBytes;
     uint64_t *full = reinterpret_cast<uint64_t *>(scl + SH::kScaleRing);
@@ -528,7 +529,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
         const int rank2 = (int)(blockIdx.x / (unsigned)p.head_groups);
         const int s2 = (p.order ? p.order[rank2] : rank2) / p.max_splits;
         merge_splits_if_last<T>(p.ws_acc, p.ws_ml, p.counters + (size_t)s2 * p.head_groups + hg2, p.out, p.out_f32,
-                                s2, p.num_q_heads, p.max_splits, nsplit, hg2 * HEADS * p.group, HEADS * p.group, kD);
+                                s2, p.num_q_heads, p.max_splits, nsplit, hg2 * HEADS * p.group, HEADS * p.group, kD,
+                                reinterpret_cast<float *>(smem), SH::kRingBytes / 4);
     }
 }
 

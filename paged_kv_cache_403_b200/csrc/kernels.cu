@@ -195,6 +195,31 @@ constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr float kRescaleThreshold = 8.0f;                // log2 units: 2^8 headroom
 
+// Split ranges.  A sequence of nblk blocks, more than split_blocks of them, is cut
+// into n = ceil(nblk / split_blocks) ranges of nearly equal length: with
+// nblk = q * n + r, the first r ranges hold q + 1 blocks and the others q, so a range
+// holds at most split_blocks blocks and, when there are several, at least
+// split_blocks / 2 (rounded down).
+// Range lengths then spread with the sequence lengths instead of piling up at
+// split_blocks, where CTAs of equal length would end (and their successors ramp up)
+// at the same moment all over the GPU.
+struct SplitRange {
+    int b0, b1, n;   // blocks [b0, b1) of range z; n ranges; b0 >= nblk when z >= n
+};
+
+__device__ __forceinline__ SplitRange split_range(int nblk, int split_blocks, int z) {
+    SplitRange r;
+    r.n = nblk > 0 ? (nblk + split_blocks - 1) / split_blocks : 0;
+    if (z >= r.n) {
+        r.b0 = r.b1 = nblk;
+        return r;
+    }
+    const int q = nblk / r.n, rem = nblk % r.n;
+    r.b0 = z * q + min(z, rem);
+    r.b1 = r.b0 + q + (z < rem ? 1 : 0);
+    return r;
+}
+
 struct DecodeParams {
     const unsigned char *k_layer;   // this layer's key pool [NB][Hkv][B][D]
     const unsigned char *v_layer;
@@ -265,11 +290,12 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_simt_kernel(const
         L = p.max_blocks * B;
     }
     const int nblk = (L + B - 1) / B;
-    const int b0 = split * p.split_blocks;
-    if (b0 >= nblk) return;
-    const int b1 = min(nblk, b0 + p.split_blocks);
+    const SplitRange rg = split_range(nblk, p.split_blocks, split);
+    if (split >= rg.n) return;
+    const int b0 = rg.b0;
+    const int b1 = rg.b1;
     const int ntiles = b1 - b0;
-    const int nsplit = (nblk + p.split_blocks - 1) / p.split_blocks;
+    const int nsplit = rg.n;
     const int group = p.num_q_heads / p.num_kv_heads;
     const int h0 = hg * HPC;
     const int g = h0 / group;
@@ -537,7 +563,8 @@ __device__ __forceinline__ int plan_bucket(const PlanParams &p, int item) {
     const int s = item / p.max_splits, z = item % p.max_splits;
     const int L = p.lens[s];
     const int nblk = L < 1 ? 0 : min((L + p.block_size - 1) / p.block_size, p.max_blocks);
-    const int t = max(0, min(p.split_blocks, nblk - z * p.split_blocks));
+    const SplitRange r = split_range(nblk, p.split_blocks, z);
+    const int t = r.b1 - r.b0;
     return kPlanBuckets - 1 - min(t, kPlanBuckets - 1);   // longest ranges in the lowest bucket
 }
 
@@ -599,7 +626,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanParams p) 
 template <typename T>
 __device__ __forceinline__ void merge_splits_if_last(const float *ws_acc, const float *ws_ml, int32_t *counter,
                                                      void *out, int out_f32, int s, int num_q_heads,
-                                                     int max_splits, int nsplit, int h0, int hpc, int D) {
+                                                     int max_splits, int nsplit, int h0, int hpc, int D,
+                                                     float *scratch, int scratch_floats) {
     __shared__ int is_last;
     __threadfence();          // this CTA's partial is visible before the count moves
     __syncthreads();
@@ -611,15 +639,81 @@ __device__ __forceinline__ void merge_splits_if_last(const float *ws_acc, const 
     __syncthreads();
     if (!is_last) return;
     __threadfence();
+    const size_t base = (size_t)s * max_splits * num_q_heads + h0;   // partial (s, split 0, head h0)
+    const int nml = nsplit * hpc;
+    if (nml * 3 + 16 <= scratch_floats && D % 4 == 0) {
+        // The partials sit in L2; every load of a phase is independent of the others,
+        // so each phase costs about one L2 round trip.  Phase 1: every (m, l) pair.
+        float *sm = scratch;              // [nsplit][hpc] running maxima
+        float *sl = sm + nml;             // [nsplit][hpc] sums
+        float *sw = sl + nml;             // [nsplit][hpc] weights 2^(m - M) / l_total
+        float *smax = sw + nml;           // [hpc] M
+        float *sinv = smax + 8;           // [hpc] 1 / l_total
+        for (int i = threadIdx.x; i < nml; i += blockDim.x) {
+            const int x = i / hpc, h = i % hpc;
+            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(ws_ml) + base + (size_t)x * num_q_heads + h);
+            sm[i] = ml.x;
+            sl[i] = ml.y;
+        }
+        __syncthreads();
+        if (threadIdx.x < hpc) {
+            const int h = threadIdx.x;
+            float mx = -INFINITY;
+            for (int x = 0; x < nsplit; ++x) mx = fmaxf(mx, sm[x * hpc + h]);
+            float lsum = 0.f;
+            for (int x = 0; x < nsplit; ++x) lsum += sl[x * hpc + h] * ex2(sm[x * hpc + h] - mx);
+            smax[h] = mx;
+            sinv[h] = 1.f / lsum;
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < nml; i += blockDim.x) {
+            const int h = i % hpc;
+            sw[i] = ex2(sm[i] - smax[h]) * sinv[h];
+        }
+        __syncthreads();
+        // Phase 2: four output columns per thread, all splits' partials loaded together.
+        const int q4 = D / 4;
+        for (int it = threadIdx.x; it < hpc * q4; it += blockDim.x) {
+            const int h = it / q4, d4 = it % q4;
+            const float4 *src = reinterpret_cast<const float4 *>(ws_acc + (base + h) * D) + d4;
+            const size_t stride = (size_t)num_q_heads * D / 4;   // float4s from one split to the next
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+            for (int x = 0; x < nsplit; ++x) {
+                const float4 a = __ldcg(src + (size_t)x * stride);
+                const float w = sw[x * hpc + h];
+                acc.x += w * a.x;
+                acc.y += w * a.y;
+                acc.z += w * a.z;
+                acc.w += w * a.w;
+            }
+            const size_t idx = ((size_t)s * num_q_heads + h0 + h) * D + 4 * d4;
+            if (out_f32) {
+                float *o = static_cast<float *>(out) + idx;
+                o[0] = acc.x;
+                o[1] = acc.y;
+                o[2] = acc.z;
+                o[3] = acc.w;
+            } else {
+                T *o = static_cast<T *>(out) + idx;
+                o[0] = Elem<T>::narrow(acc.x);
+                o[1] = Elem<T>::narrow(acc.y);
+                o[2] = Elem<T>::narrow(acc.z);
+                o[3] = Elem<T>::narrow(acc.w);
+            }
+        }
+        return;
+    }
+    // very many splits: one output element per thread, partials read split by split
     for (int t = threadIdx.x; t < hpc * D; t += blockDim.x) {
         const int h = t / D;
         const int d = t % D;
-        const size_t base = (size_t)s * max_splits * num_q_heads + h0 + h;
+        const size_t hb = base + h;
         float mx = -INFINITY;
-        for (int x = 0; x < nsplit; ++x) mx = fmaxf(mx, __ldcg(ws_ml + (base + (size_t)x * num_q_heads) * 2));
+        for (int x = 0; x < nsplit; ++x) mx = fmaxf(mx, __ldcg(ws_ml + (hb + (size_t)x * num_q_heads) * 2));
         float lsum = 0.f, osum = 0.f;
         for (int x = 0; x < nsplit; ++x) {
-            const size_t part = base + (size_t)x * num_q_heads;
+            const size_t part = hb + (size_t)x * num_q_heads;
             const float f = ex2(__ldcg(ws_ml + part * 2) - mx);
             lsum += __ldcg(ws_ml + part * 2 + 1) * f;
             osum += __ldcg(ws_acc + part * D + d) * f;
@@ -777,10 +871,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) paged_decode_mma_kernel(con
         L = p.max_blocks * B;
     }
     const int nblk = (L + B - 1) / B;
-    const int b0 = split * p.split_blocks;
-    if (b0 >= nblk) return;
-    const int ntiles = min(nblk, b0 + p.split_blocks) - b0;
-    const int nsplit = (nblk + p.split_blocks - 1) / p.split_blocks;
+    const SplitRange rg = split_range(nblk, p.split_blocks, split);
+    if (split >= rg.n) return;
+    const int b0 = rg.b0;
+    const int ntiles = rg.b1 - rg.b0;
+    const int nsplit = rg.n;
     const int group = p.num_q_heads / p.num_kv_heads;
     const int h0 = hg * hpc;
     const int g = h0 / group;
@@ -1003,7 +1098,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) paged_decode_mma_kernel(con
     }
     if (nsplit > 1)
         merge_splits_if_last<T>(p.ws_acc, p.ws_ml, p.counters + (size_t)s * p.head_groups + hg, p.out, p.out_f32, s,
-                                p.num_q_heads, p.max_splits, nsplit, h0, hpc, D);
+                                p.num_q_heads, p.max_splits, nsplit, h0, hpc, D, reinterpret_cast<float *>(smem),
+                                SH::kRingBytes / 4);
 }
 
 #include "prefill.cuh"
