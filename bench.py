@@ -133,6 +133,13 @@ def make_recipe(workload, seed_offset, steps):
     return wl.prefix_sharing(seed=4 + seed_offset)
 
 
+# Workloads whose KV (or unique KV) per step fits in the 126 MB L2: each step starts by
+# overwriting a buffer twice the L2's size, so no step finds the previous step's blocks
+# in L2.  Reuse inside one launch (a shared prefix read by many sequences) stays.
+L2_RESIDENT = ("worked_example", "prefix_sharing", "shared_prompt")
+FLUSH_BYTES = 256 << 20
+
+
 def describe(workload):
     return {
         "continuous_batch": "continuous_batch: 256 seqs, lengths U[128,4096], block 16, 32 q / 8 KV heads, d128, "
@@ -224,6 +231,29 @@ def replica_seed(rank: int) -> int:
     return 100 * rank
 
 
+# ---------------------------------------------------------------------------- staging
+class Packed:
+    """Byte layout of several arrays in one buffer, each starting on a 256-byte
+    boundary, so that one copy moves them all.  parts: (name, torch dtype, shape)."""
+
+    ALIGN = 256
+
+    def __init__(self, parts):
+        self.parts, off = [], 0
+        for name, dtype, shape in parts:
+            count = int(np.prod(shape)) if len(shape) else 1
+            nbytes = count * dtype.itemsize
+            self.parts.append((name, dtype, tuple(shape), off, nbytes))
+            off = -(-(off + nbytes) // self.ALIGN) * self.ALIGN
+        self.nbytes = max(off, self.ALIGN)
+        self.off = {name: o for name, _, _, o, _ in self.parts}
+        self.end = {name: o + nb for name, _, _, o, nb in self.parts}
+
+    def views(self, buf):
+        """name -> view of buf (a uint8 tensor of at least nbytes) with the part's dtype and shape."""
+        return {name: buf[o:o + nb].view(dt).view(shape) for name, dt, shape, o, nb in self.parts}
+
+
 # ---------------------------------------------------------------------------- our path
 class Replica:
     """One GPU's decode state: pools, block manager, sequences, and every step's inputs
@@ -289,6 +319,10 @@ class Replica:
             self.plan = static_plan(range(n), lens, total_steps)
             self.max_blocks = -(-(max(lens) + total_steps + 1) // sh.block_size)
         self.n = n
+        # sequence ids as a ready int32 array (and the one-token counts): the per-step
+        # reservation and table calls then pass pointers without converting lists
+        self.sid_arr = np.asarray(self.sids, np.int32)
+        self.ones = np.ones(n, np.int32)
         # every step's inputs (all layers), generated on the device before any timing
         self.inputs = []
         for st in self.plan:
@@ -307,33 +341,54 @@ class Replica:
                 per_layer.append((q, k, v, pk, pv))
             self.inputs.append(per_layer)
         torch.cuda.synchronize()
-        self.host = {}
-        if e2e_from is not None:      # pinned host copies for the end-to-end leg
+        # end-to-end leg: each (step, layer)'s q, K, V rows and prompt rows packed in one
+        # pinned host buffer; one copy per layer uploads them into a device buffer of the
+        # same layout (prompt rows right after the step's own rows, so only the rows of
+        # this step's admissions cross the bus)
+        self.host, self.e2e_views, self.e2e_bytes = {}, {}, {}
+        dt = self.inputs[0][0][0].dtype
+        row_shape = lambda rows: (rows, sh.num_kv_heads, sh.head_dim)  # noqa: E731
+        self.e2e_layout = {}
+        if e2e_from is not None:
             for t in range(e2e_from, total_steps):
-                self.host[t] = [[None if x is None else x.cpu().pin_memory() for x in lay]
-                                for lay in self.inputs[t]]
+                ptot_t = 0 if self.inputs[t][0][3] is None else self.inputs[t][0][3].shape[0]
+                lay = Packed([("q", dt, (n, sh.num_q_heads, sh.head_dim)), ("k", dt, row_shape(n)),
+                              ("v", dt, row_shape(n)), ("pk", dt, row_shape(ptot_t)), ("pv", dt, row_shape(ptot_t))])
+                self.e2e_layout[t] = lay
+                self.host[t] = []
+                for src in self.inputs[t]:
+                    buf = torch.empty(lay.nbytes, dtype=torch.uint8).pin_memory()
+                    views = lay.views(buf)
+                    for name, x in zip(("q", "k", "v", "pk", "pv"), src):
+                        if x is not None:
+                            views[name].copy_(x)
+                    self.host[t].append(buf)
+                self.e2e_bytes[t] = lay.end["pv"]
         mb = self.max_blocks
         pin = lambda shape, dt: torch.empty(shape, dtype=dt).pin_memory()  # noqa: E731
         max_prompt = max([sum(p - self.prompt_start(p) for _, _, p in st["admitted"]) for st in self.plan] + [1])
         H, D2 = NSETS + 1, NSETS
-        self.h_tables = [pin((n, mb), torch.int32) for _ in range(H)]
-        self.h_lens = [pin((n,), torch.int32) for _ in range(H)]
-        self.h_slots = [pin((n,), torch.int64) for _ in range(H)]
-        self.h_pslots = [pin((max_prompt,), torch.int64) for _ in range(H)]
-        self.h_cow = [pin((n, 2), torch.int32) for _ in range(H)]
+        # one step's metadata, packed so that one copy uploads it (prompt slots last: only
+        # the used ones are copied)
+        self.meta = Packed([("tables", torch.int32, (n, mb)), ("lens", torch.int32, (n,)),
+                            ("slots", torch.int64, (n,)), ("cow", torch.int32, (n, 2)),
+                            ("pslots", torch.int64, (max_prompt,))])
+        self.h_meta = [pin((self.meta.nbytes,), torch.uint8) for _ in range(H)]
+        self.d_meta = [torch.empty(self.meta.nbytes, dtype=torch.uint8, device=device) for _ in range(D2)]
+        hv = [self.meta.views(b) for b in self.h_meta]
+        dv = [self.meta.views(b) for b in self.d_meta]
+        self.h_tables, self.h_lens, self.h_slots, self.h_cow, self.h_pslots = (
+            [v[k] for v in hv] for k in ("tables", "lens", "slots", "cow", "pslots"))
+        self.d_tables, self.d_lens, self.d_slots, self.d_cow, self.d_pslots = (
+            [v[k] for v in dv] for k in ("tables", "lens", "slots", "cow", "pslots"))
         self.h_done = [None] * H
-        self.d_tables = [torch.empty((n, mb), dtype=torch.int32, device=device) for _ in range(D2)]
-        self.d_lens = [torch.empty((n,), dtype=torch.int32, device=device) for _ in range(D2)]
-        self.d_slots = [torch.empty((n,), dtype=torch.int64, device=device) for _ in range(D2)]
-        self.d_pslots = [torch.empty((max_prompt,), dtype=torch.int64, device=device) for _ in range(D2)]
-        self.d_cow = [torch.empty((n, 2), dtype=torch.int32, device=device) for _ in range(D2)]
         self.d_free = [None] * D2
-        dt = self.inputs[0][0][0].dtype
         if e2e_from is not None:
-            self.d_in = [[[torch.empty_like(x) for x in lay[:3]] for lay in self.inputs[0]] for _ in range(D2)]
-            self.d_pk = [[torch.empty((max_prompt, sh.num_kv_heads, sh.head_dim), dtype=dt, device=device)
-                          for _ in range(self.NL)] for _ in range(D2)]
-            self.d_pv = [[torch.empty_like(x) for x in self.d_pk[0]] for _ in range(D2)]
+            big = max(lay.nbytes for lay in self.e2e_layout.values())
+            self.d_in = [[torch.empty(big, dtype=torch.uint8, device=device) for _ in range(self.NL)]
+                         for _ in range(D2)]
+            for t, lay in self.e2e_layout.items():
+                self.e2e_views[t] = [lay.views(b) for b in self.d_in[t % NSETS]]
         self.out = [torch.empty((self.NL, n, sh.num_q_heads, sh.head_dim), dtype=dt, device=device)
                     for _ in range(D2)]
         self.h_out = [pin(tuple(self.out[0].shape), dt) for _ in range(D2)] if e2e_from is not None else None
@@ -345,12 +400,16 @@ class Replica:
         self.scale = 1.0 / math.sqrt(sh.head_dim)
         self.attn_events = []
         self.kv_bytes, self.alg_bytes, self.h2d, self.d2h, self.prompt_rows_appended = [], [], [], [], []
+        self.host_s = []
+        self.flush = (torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device) if workload in L2_RESIDENT
+                      else None)
 
     def step(self, t, e2e=False, time_attention=True):
         torch, pa, sh, plan = self.torch, self.pa, self.shape, self.plan[t]
         n, hs, ds = self.n, t % (NSETS + 1), t % NSETS
         if self.h_done[hs] is not None:      # staging set hs: its uploads (NSETS + 1 steps ago) are done
             self.h_done[hs].synchronize()
+        h0 = time.perf_counter()             # host work of this step, not counting that wait
         # 1. admissions: new sequences take the retired slots; their prompts are appended below
         ptot = 0
         if plan["admitted"]:
@@ -362,43 +421,34 @@ class Replica:
                 else:
                     sid = self.cache.add()
                 self.sids[slot] = sid
+                self.sid_arr[slot] = sid
                 new.append((sid, plen - self.prompt_start(plen)))
             pslots, _ = pa.pa_reserve_slots(self.cache.pool, [s for s, _ in new], [p for _, p in new],
                                             slot_out=self.h_pslots[hs])
             ptot = len(pslots)
         self.prompt_rows_appended.append(ptot)
         # 2. one slot per sequence for this step's token (new block, or copy-on-write of a shared tail)
-        _, cow = pa.pa_reserve_slots(self.cache.pool, self.sids, [1] * n, slot_out=self.h_slots[hs],
+        _, cow = pa.pa_reserve_slots(self.cache.pool, self.sid_arr, self.ones, slot_out=self.h_slots[hs],
                                      cow_out=self.h_cow[hs])
         ncow = len(cow)
-        _, lens = pa.pa_build_block_tables(self.cache.pool, self.sids, self.max_blocks, self.h_tables[hs],
+        _, lens = pa.pa_build_block_tables(self.cache.pool, self.sid_arr, self.max_blocks, self.h_tables[hs],
                                            self.h_lens[hs])
         # 3. uploads (metadata; end to end also the step's inputs) on the copy stream
         if self.d_free[ds] is not None:
             self.copy.wait_event(self.d_free[ds])
-        h2d = self.h_tables[hs].numel() * 4 + n * 4 + n * 8 + ptot * 8 + ncow * 8
+        mbytes = self.meta.off["pslots"] + ptot * 8          # everything through the used prompt slots
+        h2d = mbytes
         with torch.cuda.stream(self.copy):
-            self.d_tables[ds].copy_(self.h_tables[hs], non_blocking=True)
-            self.d_lens[ds].copy_(self.h_lens[hs], non_blocking=True)
-            self.d_slots[ds].copy_(self.h_slots[hs], non_blocking=True)
-            if ptot:
-                self.d_pslots[ds][:ptot].copy_(self.h_pslots[hs][:ptot], non_blocking=True)
-            if ncow:
-                self.d_cow[ds][:ncow].copy_(self.h_cow[hs][:ncow], non_blocking=True)
+            self.d_meta[ds][:mbytes].copy_(self.h_meta[hs][:mbytes], non_blocking=True)
             if e2e:
                 layers = []
+                nb = self.e2e_bytes[t]
                 for layer, host in enumerate(self.host[t]):
-                    q, k, v = self.d_in[ds][layer]
-                    for dst, src in ((q, host[0]), (k, host[1]), (v, host[2])):
-                        dst.copy_(src, non_blocking=True)
-                        h2d += src.numel() * src.element_size()
-                    pk = pv = None
-                    if ptot:
-                        pk, pv = self.d_pk[ds][layer][:ptot], self.d_pv[ds][layer][:ptot]
-                        pk.copy_(host[3], non_blocking=True)
-                        pv.copy_(host[4], non_blocking=True)
-                        h2d += 2 * host[3].numel() * host[3].element_size()
-                    layers.append((q, k, v, pk, pv))
+                    self.d_in[ds][layer][:nb].copy_(host[:nb], non_blocking=True)
+                    h2d += nb
+                    v = self.e2e_views[t][layer]
+                    assert v["pk"].shape[0] == ptot
+                    layers.append((v["q"], v["k"], v["v"], v["pk"] if ptot else None, v["pv"] if ptot else None))
             else:
                 layers = self.inputs[t]
             up = torch.cuda.Event()
@@ -408,6 +458,8 @@ class Replica:
         if self.out_read[ds] is not None:    # the read-back of out[ds] (NSETS steps ago) is done
             self.compute.wait_event(self.out_read[ds])
         # 4. device work
+        if self.flush is not None:           # evict the previous step's blocks from L2
+            self.flush.fill_(t & 0xFF)
         if ncow:
             pa.pa_copy_blocks(self.cache.pool, self.d_cow[ds], ncow, stream=self.compute)
         for layer, (q, k, v, pk, pv) in enumerate(layers):
@@ -447,6 +499,7 @@ class Replica:
                               + 4 * n)
         self.kv_bytes.append(kv)
         self.alg_bytes.append(alg)
+        self.host_s.append(time.perf_counter() - h0)
         self.h2d.append(h2d)
         self.d2h.append(d2h)
 
@@ -489,6 +542,7 @@ def run_ours(args):
         rep.step(t, time_attention=False)
     rep.kv_bytes.clear()
     rep.alg_bytes.clear()
+    rep.host_s.clear()
     rep.prompt_rows_appended.clear()
     barrier()
     clocks = ClockSampler(local)
@@ -507,11 +561,13 @@ def run_ours(args):
     prompt_rows = sum(rep.prompt_rows_appended)
     attn_ms = [a.elapsed_time(b) for a, b in rep.attn_events]
     alg_per_launch = sum(rep.alg_bytes) / (K * rep.NL)
+    host_ms = 1e3 * sum(rep.host_s) / K
 
     e2e_ms = e2e_kv = 0.0
     e2e_io = (0, 0)
     if e2e:
         rep.kv_bytes.clear()
+        rep.host_s.clear()
         rep.h2d.clear()
         rep.d2h.clear()
         barrier()
@@ -524,6 +580,7 @@ def run_ours(args):
         t1.record(rep.compute)
         barrier()
         e2e_ms, e2e_kv = t0.elapsed_time(t1), sum(rep.kv_bytes)
+        e2e_host_ms = 1e3 * sum(rep.host_s) / K
         e2e_io = (sum(rep.h2d) / K, sum(rep.d2h) / K)
     clk = clocks.stop()
 
@@ -554,7 +611,10 @@ def run_ours(args):
                        "parallelism": f"replicas x{world}",
                        "kv_cache": ("E4M3 codes + one power-of-two scale byte per (token, KV head) row"
                                     if rep.kv_fp8 else sh.dtype),
-                       "l2": "no flush: the KV read per step exceeds the 126 MB L2"},
+                       "l2": (f"flushed: every step first writes {FLUSH_BYTES >> 20} MiB on the compute stream "
+                              "(inside the step time, outside the attention events)"
+                              if rep.flush is not None else
+                              "no flush: the KV read per step exceeds the 126 MB L2")},
             "decode_tokens_per_s": round(world * rep.n * K / (ms * 1e-3), 1),
             "kv_gb_per_step": round(kv_tot / K / 1e9 / world, 4),
             "hbm_fraction_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
@@ -567,6 +627,8 @@ def run_ours(args):
                          "attn_ms_mean": round(attn_mean_ms, 4), "alg_bytes_per_launch": int(alg_per_launch),
                          "launches_timed": len(attn_ms), "peak_source": peak_src},
             "gpu_launches": int(launches),
+            "host_ms_per_step": round(host_ms, 4),
+            "device_error": pa.pa_device_error(),
             "clocks": clk,
         }
         stats = rep.pa.pa_pool_stats(rep.cache.pool)
@@ -580,13 +642,19 @@ def run_ours(args):
         if e2e:
             line["e2e"] = {"value": round(e2e_kv / (e2e_ms * 1e-3) / 1e9, 1), "unit": UNIT,
                            "h2d_bytes_per_step": int(e2e_io[0]), "d2h_bytes_per_step": int(e2e_io[1]),
-                           "ms_per_step": round(e2e_ms / K, 4)}
+                           "ms_per_step": round(e2e_ms / K, 4), "host_ms_per_step": round(e2e_host_ms, 4)}
         if not args.no_cpu_baseline and args.workload not in ("prefix_sharing", "shared_prompt") and not rep.kv_fp8:
             line["cpu_baseline"] = cpu_baseline(rep, args.cpu_sample_seqs, W, args.cpu_seconds)
         print(json.dumps(line), flush=True)
+        if line["device_error"]:
+            print(f"bench.py: the kernels reported device error word {line['device_error']:#x}; "
+                  "the figures above are not of a valid run", file=sys.stderr)
+    bad = rank == 0 and bool(line["device_error"])
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    if bad:
+        raise SystemExit(1)
 
 
 # ---------------------------------------------------------------------------- oracle (CPU)
@@ -622,8 +690,9 @@ def oracle_sample(recipe, plan_step, picks, layer=0):
             np.array(lens, np.int32), np.stack(qs))
 
 
-def time_oracle(recipe, plan_step, picks, min_seconds=0.0, max_reps=1000):
-    """Runs the oracle (as it stands) on the sample, repeated until min_seconds have passed."""
+def time_oracle(recipe, plan_step, picks, min_seconds=0.0, max_reps=1000, n_threads=0):
+    """Runs the oracle (as it stands) on the sample, repeated until min_seconds have passed
+    (n_threads 0: every host core)."""
     import oracle
     sh = recipe["shape"]
     k, v, tables, lens, q = oracle_sample(recipe, plan_step, picks)
@@ -631,7 +700,7 @@ def time_oracle(recipe, plan_step, picks, min_seconds=0.0, max_reps=1000):
     reps, dt = 0, 0.0
     while reps < max_reps and (reps == 0 or dt < min_seconds):
         t0 = time.perf_counter()
-        oracle.paged_decode(k, v, sh.dtype, tables, lens, q, 1.0 / math.sqrt(sh.head_dim))
+        oracle.paged_decode(k, v, sh.dtype, tables, lens, q, 1.0 / math.sqrt(sh.head_dim), n_threads)
         dt += time.perf_counter() - t0
         reps += 1
     return kv1 * reps, dt, reps, kv1
@@ -641,11 +710,14 @@ def cpu_baseline(rep, nseq, step, seconds):
     import oracle
     picks = list(range(0, rep.n, max(1, rep.n // nseq)))[:nseq]
     kv, dt, reps, kv1 = time_oracle(rep.recipe, rep.plan[step], picks, min_seconds=seconds)
+    kv_1, dt_1, _, _ = time_oracle(rep.recipe, rep.plan[step], picks, min_seconds=seconds / 4, n_threads=1)
     layers = f"; 1 of {rep.NL} layers" if rep.NL > 1 else ""
     return {"value": round(kv / dt / 1e9, 4), "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "value_1_thread": round(kv_1 / dt_1 / 1e9, 4),
             "sample": f"fp64 oracle attention for {len(picks)} of {rep.n} sequences of one decode step "
                       f"({kv1 / 1e6:.1f} MB of KV{layers}), repeated {reps}x for {dt:.1f} s; "
-                      "OpenMP over (sequence, head)"}
+                      f"OpenMP over (sequence, head); value_1_thread: the same sample on one thread "
+                      f"for {dt_1:.1f} s"}
 
 
 def run_reference(args):

@@ -1,0 +1,62 @@
+"""Host-side staging of bench.py on CPU: the packed layouts that let one copy upload a
+step's metadata (and, end to end, a layer's q/K/V and prompt rows)."""
+import numpy as np
+import torch
+
+import bench
+
+
+def _meta(n=5, mb=7, max_prompt=11):
+    return bench.Packed([("tables", torch.int32, (n, mb)), ("lens", torch.int32, (n,)),
+                         ("slots", torch.int64, (n,)), ("cow", torch.int32, (n, 2)),
+                         ("pslots", torch.int64, (max_prompt,))])
+
+
+def test_parts_are_aligned_disjoint_and_in_order():
+    m = _meta()
+    prev_end = 0
+    for name, dt, shape, off, nbytes in m.parts:
+        assert off % bench.Packed.ALIGN == 0 and off >= prev_end
+        assert nbytes == int(np.prod(shape)) * dt.itemsize
+        prev_end = off + nbytes
+    assert m.nbytes >= prev_end and m.nbytes % bench.Packed.ALIGN == 0
+
+
+def test_views_have_the_part_shapes_and_write_through():
+    m = _meta()
+    buf = torch.zeros(m.nbytes, dtype=torch.uint8)
+    v = m.views(buf)
+    assert v["tables"].shape == (5, 7) and v["tables"].dtype == torch.int32 and v["tables"].is_contiguous()
+    assert v["cow"].shape == (5, 2) and v["pslots"].dtype == torch.int64
+    v["tables"][:] = torch.arange(35, dtype=torch.int32).view(5, 7)
+    v["pslots"][:3] = torch.tensor([7, -1, 1 << 40])
+    w = m.views(buf.clone())
+    assert torch.equal(w["tables"], v["tables"]) and w["pslots"][:3].tolist() == [7, -1, 1 << 40]
+
+
+def test_one_prefix_copy_carries_every_part_and_the_used_prompt_slots():
+    m = _meta()
+    host = torch.zeros(m.nbytes, dtype=torch.uint8)
+    hv = m.views(host)
+    rng = np.random.default_rng(0)
+    for name in ("tables", "lens", "slots", "cow", "pslots"):
+        hv[name].copy_(torch.from_numpy(rng.integers(-9, 1 << 20, hv[name].shape).astype(
+            np.int64 if hv[name].dtype == torch.int64 else np.int32)))
+    ptot = 4
+    nb = m.off["pslots"] + ptot * 8
+    dev = torch.full((m.nbytes,), 0xEE, dtype=torch.uint8)
+    dev[:nb].copy_(host[:nb])
+    dv = m.views(dev)
+    for name in ("tables", "lens", "slots", "cow"):
+        assert torch.equal(dv[name], hv[name])
+    assert torch.equal(dv["pslots"][:ptot], hv["pslots"][:ptot])
+    assert not torch.equal(dv["pslots"][ptot:], hv["pslots"][ptot:])   # unused slots were not copied
+
+
+def test_empty_prompt_part():
+    p = bench.Packed([("q", torch.bfloat16, (4, 2, 8)), ("pk", torch.bfloat16, (0, 2, 8)),
+                      ("pv", torch.bfloat16, (0, 2, 8))])
+    v = p.views(torch.zeros(p.nbytes, dtype=torch.uint8))
+    assert v["pk"].shape == (0, 2, 8) and v["pv"].numel() == 0
+    assert p.end["q"] == 4 * 2 * 8 * 2 and p.off["pk"] == bench.Packed.ALIGN
+    assert p.end["pv"] == p.off["pv"] == p.off["pk"]
