@@ -250,6 +250,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
         // ---------------- producer
         const int32_t *trow = p.tables + (size_t)s * p.max_blocks + b0;
         bool ok = true;
+        int issued = 0;
         for (int base = 0; base < ntiles && ok; base += 32) {
             int blk = 0;
             if (base + lane < ntiles) {
@@ -274,12 +275,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
                         tma_load_2d(dst, &p.tmap_k, 0, row, &full[st]);
                         tma_load_2d(dst + TILE, &p.tmap_v, 0, row, &full[st]);
                         bulk_g2s(scl + st * SCB, p.s_layer + hb0 * 2 * B, SCB, &full[st]);
+                        issued = i + 1;
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
             }
         }
+        if (lane == 0) drain_copies(full, issued, STAGES);
+        __syncwarp();
     } else {
         // ---------------- consumers
         // Q^T fragments: column gq is query head h0 + gq; lane (gq, tq) holds dims

@@ -105,6 +105,16 @@ __device__ __forceinline__ bool mbar_wait_thread(uint64_t *bar, uint32_t parity)
     return true;
 }
 
+// Before its ring is reused or the CTA exits, the issuing lane waits (bounded) until
+// the last copy it put into each stage has landed: fill i went to stage i % stages as
+// that stage's phase i / stages, and only the last `stages` fills can still be in
+// flight.  In a normal run they landed long before; after a consumer gave up on a
+// wait this keeps a late copy from writing into shared memory that is reused.
+__device__ __forceinline__ void drain_copies(uint64_t *full, int issued, int stages) {
+    for (int i = issued > stages ? issued - stages : 0; i < issued; ++i)
+        if (!mbar_wait_thread(&full[i % stages], (uint32_t)(i / stages) & 1u)) return;
+}
+
 // A whole warp waits and leaves together, so later full-warp shuffles stay converged.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity) {
     uint64_t t0 = 0;
@@ -321,6 +331,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_simt_kernel(const
         // ---------------- producer: walk the table, keep the ring full
         const int32_t *trow = p.tables + (size_t)s * p.max_blocks + b0;
         bool ok = true;
+        int issued = 0;
         for (int base = 0; base < ntiles && ok; base += 32) {
             int blk = 0;
             if (base + lane < ntiles) {
@@ -343,12 +354,15 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_simt_kernel(const
                         mbar_arrive_expect_tx(&full[st], 2 * TILE);
                         bulk_g2s(dst, p.k_layer + off, TILE, &full[st]);
                         bulk_g2s(dst + TILE, p.v_layer + off, TILE, &full[st]);
+                        issued = i + 1;
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
             }
         }
+        if (lane == 0) drain_copies(full, issued, STAGES);
+        __syncwarp();
     } else {
         // ---------------- consumers
         const int c = lane % kLanesPerToken;       // which 16-byte chunks of the row
@@ -906,6 +920,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) paged_decode_mma_kernel(con
         // ---------------- producer
         const int32_t *trow = p.tables + (size_t)s * p.max_blocks + b0;
         bool ok = true;
+        int issued = 0;
         for (int base = 0; base < ntiles && ok; base += 32) {
             int blk = 0;
             if (base + lane < ntiles) {
@@ -931,12 +946,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) paged_decode_mma_kernel(con
                             tma_load_2d(dst + bx * BOX, &p.tmap_k, bx * 64, row, &full[st]);
                             tma_load_2d(dst + TILE + bx * BOX, &p.tmap_v, bx * 64, row, &full[st]);
                         }
+                        issued = i + 1;
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
             }
         }
+        if (lane == 0) drain_copies(full, issued, STAGES);
+        __syncwarp();
     } else {
         // ---------------- consumers
         uint32_t qb[KD][2];   // Q^T fragments: column gq is query head h0 + gq

@@ -290,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
     if (warp == kTmaWarp) {
         // ---------------- producer: walk the table, keep the ring full
         const int32_t *trow = p.tables + (size_t)s * p.max_blocks;
+        int issued_k = 0, issued_v = 0;   // tiles whose K / V copies were issued
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j % kStages;
             int blk = 0;
@@ -317,10 +318,20 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                                         kv == 0 ? &p.tmap_k : &p.tmap_v, h * 64, r0, full);
                     }
                 }
+                if (kv == 0)
+                    issued_k = j + 1;
+                else
+                    issued_v = j + 1;
             }
             if (*abort_flag) break;
             __syncwarp();
         }
+        // every issued copy lands before the CTA frees its shared memory, also after an abort
+        if (lane == 0) {
+            drain_copies(k_full, issued_k, kStages);
+            drain_copies(v_full, issued_v, kStages);
+        }
+        __syncwarp();
     } else if (warp == kMmaWarp) {
         // ---------------- tensor-core issue
         // wait for tile j's keys
