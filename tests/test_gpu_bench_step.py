@@ -4,7 +4,7 @@ The benchmark drives the library through its own step: packed metadata uploads o
 side copy stream, four rotating device buffer sets, host bookkeeping running ahead of
 the GPU, and an end-to-end leg whose inputs come from pinned host memory in one packed
 copy per layer and whose output is read back on a third stream.  These tests run that
-step on the continuous-batch workload (bf16 and FP8 caches, split 2048 as timed) and
+step on the continuous-batch workload (bf16 and FP8 caches, at the splits it times) and
 compare sampled outputs of both legs with the fp64 oracle over regenerated histories.
 """
 import numpy as np
@@ -33,7 +33,8 @@ def test_bench_step_matches_oracle(kv_fp8):
     pa.pa_device_error(clear=True)
     recipe = bench.make_recipe("continuous_batch", bench.replica_seed(0), total)
     sh = recipe["shape"]
-    rep = bench.Replica(torch, "continuous_batch", recipe, total, 2048, torch.device("cuda", 0), W + K,
+    split = bench.default_split("continuous_batch")
+    rep = bench.Replica(torch, "continuous_batch", recipe, total, split, torch.device("cuda", 0), W + K,
                         kv_fp8=kv_fp8)
     for t in range(W + K):
         rep.step(t)

@@ -326,10 +326,12 @@ def test_fp8_pool_rejections():
 
 # ------------------------------------------------------------------ full sizes
 @pytest.mark.slow
-def test_continuous_batch_fp8_full_size_sampled():
-    """256 sequences, 64 steps, FP8 cache, bf16 output, split 2048 as the benchmark times
-    them; sampled sequences against the oracle over their regenerated, oracle-quantised
-    histories, and sampled cache rows bit-exact against the oracle's quantiser."""
+@pytest.mark.parametrize("split", [2048, 4096])
+def test_continuous_batch_fp8_full_size_sampled(split):
+    """256 sequences, 64 steps, FP8 cache, bf16 output, split 4096 (the benchmark's
+    default) and 2048; sampled sequences against the oracle
+    over their regenerated, oracle-quantised histories, and sampled cache rows bit-exact
+    against the oracle's quantiser."""
     from oracle_replay import sequence_attention_fp8
     from paged_kv_cache_403_b200.runners import ContinuousBatch
     from synthetic import workloads as wl
@@ -338,7 +340,7 @@ def test_continuous_batch_fp8_full_size_sampled():
     cb = ContinuousBatch(r, kv_fp8=True)
     rng = np.random.default_rng(0)
     for t in range(64):
-        rec = cb.step(split_tokens=2048)
+        rec = cb.step(split_tokens=split)
         if t in (0, 33, 63):
             lens = rec.lens
             picks = set(rng.choice(len(lens), size=5, replace=False).tolist())
@@ -358,15 +360,16 @@ def test_continuous_batch_fp8_full_size_sampled():
 
 
 @pytest.mark.slow
-def test_large_pool_fp8_sampled():
-    """384 sequences, lognormal lengths, 32 layers, block 32, FP8 cache (~50 GB), split 2048
-    as the benchmark times it; layers 0 and 31 sampled against the oracle."""
+@pytest.mark.parametrize("split", [2048, 4096])
+def test_large_pool_fp8_sampled(split):
+    """384 sequences, lognormal lengths, 32 layers, block 32, FP8 cache (~50 GB), split 4096
+    (the benchmark's default) and 2048; layers 0 and 31 sampled against the oracle."""
     from oracle_replay import sequence_attention_fp8
     from paged_kv_cache_403_b200.runners import run_static
     from synthetic import workloads as wl
     r = wl.large_pool(block_size=32)
     sh = r["shape"]
-    cache, _, rec = run_static(r, split_tokens=2048, keep_layers={0, 31}, kv_fp8=True)
+    cache, _, rec = run_static(r, split_tokens=split, keep_layers={0, 31}, kv_fp8=True)
     lens = rec.lens
     picks = [int(np.argmax(lens)), int(np.argmin(lens)), int(np.argsort(lens)[len(lens) // 2])]
     picks += [int(i) for i in np.nonzero(lens > 4096)[0][:2]]

@@ -180,15 +180,16 @@ def test_continuous_batch_reduced_full_replay():
 
 
 @pytest.mark.slow
-def test_continuous_batch_full_size_sampled():
-    """256 sequences, 64 steps, bf16 output, split 2048 as timed by the benchmark;
-    sampled sequences checked against the oracle on regenerated histories."""
+@pytest.mark.parametrize("split", [2048, 4096])
+def test_continuous_batch_full_size_sampled(split):
+    """256 sequences, 64 steps, bf16 output, split 4096 as timed by the benchmark (and
+    2048); sampled sequences checked against the oracle on regenerated histories."""
     r = wl.continuous_batch()
     sh = r["shape"]
     cb = ContinuousBatch(r)
     rng = np.random.default_rng(0)
     for t in range(64):
-        rec = cb.step(split_tokens=2048)
+        rec = cb.step(split_tokens=split)
         if t in (0, 21, 63):
             lens = rec.lens
             picks = set(rng.choice(len(lens), size=5, replace=False).tolist())
@@ -208,10 +209,11 @@ def test_continuous_batch_full_size_sampled():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("bs,split", [(16, 2048), (32, 2048), (16, 4096)])
+@pytest.mark.parametrize("bs,split", [(16, 2048), (32, 2048), (16, 4096), (32, 4096)])
 def test_large_pool_sampled(bs, split):
-    """384 sequences, lognormal lengths, 32 layers (~100 GB), split-K: 2048-token ranges as
-    the benchmark times them, and 4096 (split only sequences over 4096 tokens)."""
+    """384 sequences, lognormal lengths, 32 layers (~100 GB), split-K: ranges of at most
+    4096 tokens as the benchmark times them (only sequences over 4096 tokens split), and
+    2048."""
     r = wl.large_pool(block_size=bs)
     sh = r["shape"]
     cache, _, rec = run_static(r, split_tokens=split, keep_layers={0, 31})
