@@ -100,3 +100,18 @@ def test_decode_workspace_sizes_cover_every_part():
         order = -(-(n * ms * 4) // 16) * 16
         counters = -(-(n * hq * 4) // 16) * 16 if ms > 1 else 0
         assert pa.pa_decode_workspace_bytes(n, hq, d, ms) == partials + order + counters
+
+
+def test_static_entry_limit_matches_header_and_refuses_oversize_batches_before_any_device_call():
+    text = open(os.path.join(ROOT, "include", "pa.h")).read()
+    m = re.search(r"#define PA_STATIC_WORKSPACE_BYTES \((\d+)u << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == pa.PA_STATIC_WORKSPACE_BYTES
+    # 4096 sequences of 32 q heads, 17 split ranges each: partials far beyond the array
+    pool = pa.pa_pool_create(1, 8, 16, 8, 128, "bf16")
+    ms = pa.pa_decode_max_splits(16, 4096 // 16 + 1, 256)
+    assert pa.pa_decode_workspace_bytes(4096, 32, 128, ms) > pa.PA_STATIC_WORKSPACE_BYTES
+    st = pa._lib().pa_decode_attention_static(pool, 0, None, None, 2, None, 4096 // 16 + 1, None, 4096, 32,
+                                             0.1, 256, None)
+    assert st == pa.PA_ERR_INVALID_ARG
+    assert "split scratch" in pa.pa_last_error() and str(pa.PA_STATIC_WORKSPACE_BYTES) in pa.pa_last_error()
+    pa.pa_pool_destroy(pool)
