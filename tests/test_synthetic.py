@@ -49,3 +49,41 @@ def test_workload_sizes():
     # about 100 GB of fp16 cache at 128 KiB per token
     assert 80e9 < tokens * 131072 < 130e9
     assert abs(math.log(np.median(lp["lens"])) - math.log(1500)) < 0.15
+
+
+def test_continuous_schedule_stop_rate_and_replacements():
+    """Stops are independent Bernoulli(1/200) per sequence and step; replacements draw
+    U[128, 4096]: over 64 steps x 256 slots the stop count sits within 4 sigma of 81.92."""
+    s = wl.continuous_schedule(256, 64, seed=3)
+    stops = [e for ev in s.events for e in ev]
+    mean, sd = 256 * 64 / 200, math.sqrt(256 * 64 * (1 / 200) * (199 / 200))
+    assert abs(len(stops) - mean) < 4 * sd
+    assert all(0 <= slot < 256 and 128 <= plen <= 4096 for slot, plen in stops)
+    for ev in s.events:                   # ascending slot order, each slot at most once per step
+        slots = [slot for slot, _ in ev]
+        assert slots == sorted(set(slots))
+    big = wl.continuous_schedule(256, 2000, seed=11)
+    rate = sum(len(ev) for ev in big.events) / (256 * 2000)
+    assert abs(rate - 1 / 200) < 4 * math.sqrt((1 / 200) * (199 / 200) / (256 * 2000))
+
+
+def test_benchmark_plan_follows_the_schedule():
+    """The benchmark's step plan: batch size fixed, continuing sequences grow by one token
+    a step, a retired slot is taken at the next step by a new uid at its prompt length."""
+    import bench
+    r = wl.continuous_batch(seed=3, steps=40, p_stop=0.05)
+    sched = r["schedule"]
+    plan = bench.simulate(sched, 256, 40)
+    assert np.array_equal(plan[0]["pos"], sched.initial) and np.array_equal(plan[0]["uids"], np.arange(256))
+    next_uid = 256
+    for t in range(1, 40):
+        prev, cur = plan[t - 1], plan[t]
+        retired = {slot: plen for slot, plen in sched.events[t - 1]}
+        assert [a[0] for a in cur["admitted"]] == sorted(retired)
+        for slot, uid, plen in cur["admitted"]:
+            assert uid == next_uid and plen == retired[slot] and cur["pos"][slot] == plen
+            next_uid += 1
+        keep = np.array([i not in retired for i in range(256)])
+        assert np.array_equal(cur["pos"][keep], prev["pos"][keep] + 1)
+        assert np.array_equal(cur["uids"][keep], prev["uids"][keep])
+        assert cur["retire"] == list(sched.events[t])
