@@ -328,6 +328,7 @@ pa_status pa_reserve_slots(pa_pool *p, const int32_t *seq_ids, const int32_t *nt
         return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: bad argument");
     int64_t total = 0;
     std::vector<pa_pool::Seq *> seqs((size_t)n);
+    const uint64_t call = ++p->batch_calls;   // a sequence listed twice in this call is seen twice
     for (int32_t i = 0; i < n; ++i) {
         auto it = p->seqs.find(seq_ids[i]);
         if (it == p->seqs.end() || ntok[i] < 0)
@@ -335,19 +336,16 @@ pa_status pa_reserve_slots(pa_pool *p, const int32_t *seq_ids, const int32_t *nt
         if (it->second.swapped) return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: sequence is swapped out");
         if ((int64_t)it->second.len + ntok[i] > INT32_MAX)
             return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: sequence too long");
+        if (it->second.seen == call) return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: duplicate sequence id");
+        it->second.seen = call;
         seqs[i] = &it->second;
         total += ntok[i];
-    }
-    {   // distinct ids
-        std::vector<int32_t> ids(seq_ids, seq_ids + n);
-        std::sort(ids.begin(), ids.end());
-        if (std::adjacent_find(ids.begin(), ids.end()) != ids.end())
-            return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: duplicate sequence id");
     }
     if (total > 0 && !slot_mapping_out) return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: null slot_mapping_out");
 
     const int32_t B = p->cfg.block_size;
     std::vector<Undo> journal;
+    journal.reserve((size_t)total + 16);   // one length record per token, more only at block boundaries
     int32_t cows = 0;
     int64_t k = 0;
     pa_status st = PA_OK;

@@ -25,9 +25,11 @@ struct pa_pool {
         std::vector<int32_t> table;   // logical block -> physical block
         int32_t len = 0;              // tokens
         bool swapped = false;         // blocks live in host memory (pa_swap_out)
+        uint64_t seen = 0;            // last batch call that listed this sequence
     };
     std::unordered_map<int32_t, Seq> seqs;
     int32_t next_seq = 0;
+    uint64_t batch_calls = 0;         // numbers batch calls, for the duplicate-id check
 
     int64_t num_tokens = 0;
     int64_t cow_copies = 0;

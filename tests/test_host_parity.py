@@ -269,3 +269,19 @@ def test_invalid_arguments_rejected():
     t, ln = pa.pa_build_block_tables(p, [s], 5)
     assert ln.tolist() == [40] and t[0, 3:].tolist() == [-1, -1]
     pa.pa_pool_destroy(p)
+
+
+def test_duplicate_ids_rejected_without_change_and_next_call_unaffected():
+    p = pa.pa_pool_create(1, 8, 16, 1, 64, "f16")
+    a, b = pa.pa_seq_add(p), pa.pa_seq_add(p)
+    pa.pa_reserve_slots(p, [a, b], [3, 5])
+    free_before = pa.pa_free_list(p).tolist()
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_reserve_slots(p, [a, b, a], [1, 1, 1])
+    assert e.value.status == pa.PA_ERR_INVALID_ARG and "duplicate" in str(e.value)
+    assert pa.pa_seq_info(p, a)[0] == 3 and pa.pa_seq_info(p, b)[0] == 5
+    assert pa.pa_free_list(p).tolist() == free_before
+    slots, _ = pa.pa_reserve_slots(p, [b, a], [1, 1])     # the same ids again, once each
+    ta, tb = pa.pa_seq_info(p, a)[1], pa.pa_seq_info(p, b)[1]
+    assert slots.tolist() == [int(tb[0]) * 16 + 5, int(ta[0]) * 16 + 3]
+    pa.pa_pool_destroy(p)
