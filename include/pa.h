@@ -279,8 +279,10 @@ size_t pa_decode_workspace_bytes(int32_t n_seqs, int32_t num_q_heads, int32_t he
  * out_dtype (PA_F32 or the pool dtype / act_dtype); block_tables_dev [n_seqs][max_blocks]
  * int32, seq_lens_dev [n_seqs] int32 >= 1, all device pointers.  Sequences with
  * more than split_tokens tokens (a multiple of block_size; 0 = never) are split
- * into ranges of split_tokens whose partial results are merged (on the tensor-core
- * paths by the last CTA of each range, on the fp32 path by a second kernel); that needs
+ * into ceil(blocks / (split_tokens / block_size)) ranges of nearly equal length (at
+ * most split_tokens tokens each, the first ones one block longer) whose partial
+ * results are merged (on the tensor-core paths by the last CTA of each range, on
+ * the fp32 path by a second kernel); that needs
  * `workspace` of pa_decode_workspace_bytes(n_seqs, num_q_heads, head_dim,
  * pa_decode_max_splits(...)) bytes (caller-owned device memory, 16-byte aligned,
  * contents need not be initialised).  With a workspace of that size the call first
