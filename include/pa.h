@@ -50,7 +50,8 @@ typedef enum {
     PA_ERR_OUT_OF_BLOCKS = 2,  /* the free list cannot satisfy the call */
     PA_ERR_DOUBLE_FREE = 3,    /* a block with refcount 0 was freed */
     PA_ERR_CUDA = 4,           /* a CUDA runtime call or kernel launch failed */
-    PA_ERR_UNSUPPORTED = 5     /* a valid shape the kernels are not built for */
+    PA_ERR_UNSUPPORTED = 5,    /* a valid shape the kernels are not built for */
+    PA_ERR_HOST_MEMORY = 6     /* host memory for the block manager's own records ran out */
 } pa_status;
 
 /* PA_FP8_E4M3 is a cache storage type only: see "FP8 cache" below. */
@@ -175,7 +176,10 @@ pa_status pa_seq_info(const pa_pool *pool, int32_t seq_id, int32_t *len, int32_t
  * Outputs (host buffers): slot_mapping_out[sum(ntok)] in batch order;
  * cow_pairs_out[2 * k] = (src, dst) for each copy, at most n pairs (one per
  * sequence); *n_cow = k.  seq_ids must be distinct.  On PA_ERR_OUT_OF_BLOCKS
- * nothing changes.  The caller copies the pairs to the device and calls
+ * nothing changes; a call whose block-boundary crossings alone need more blocks
+ * than are free (or evictable) fails that way before anything is taken, whatever
+ * the counts.  PA_ERR_HOST_MEMORY (the host could not grow the call's own records)
+ * also leaves everything unchanged.  The caller copies the pairs to the device and calls
  * pa_copy_blocks before writing the new tokens with pa_append_kv. */
 pa_status pa_reserve_slots(pa_pool *pool, const int32_t *seq_ids, const int32_t *ntok, int32_t n,
                            int64_t *slot_mapping_out, int32_t *cow_pairs_out, int32_t *n_cow);

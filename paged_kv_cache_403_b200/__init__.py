@@ -14,7 +14,8 @@ import numpy as np
 from . import _native
 from ._native import PoolConfig, PoolStats
 
-PA_OK, PA_ERR_INVALID_ARG, PA_ERR_OUT_OF_BLOCKS, PA_ERR_DOUBLE_FREE, PA_ERR_CUDA, PA_ERR_UNSUPPORTED = range(6)
+(PA_OK, PA_ERR_INVALID_ARG, PA_ERR_OUT_OF_BLOCKS, PA_ERR_DOUBLE_FREE, PA_ERR_CUDA, PA_ERR_UNSUPPORTED,
+ PA_ERR_HOST_MEMORY) = range(7)
 PA_F32, PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2, 3
 DTYPE_CODES = {"f32": PA_F32, "f16": PA_F16, "bf16": PA_BF16, "fp8": PA_FP8_E4M3}
 
@@ -23,7 +24,7 @@ class PaError(RuntimeError):
     def __init__(self, status: int, message: str):
         self.status = status
         names = {1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_OUT_OF_BLOCKS", 3: "PA_ERR_DOUBLE_FREE",
-                 4: "PA_ERR_CUDA", 5: "PA_ERR_UNSUPPORTED"}
+                 4: "PA_ERR_CUDA", 5: "PA_ERR_UNSUPPORTED", 6: "PA_ERR_HOST_MEMORY"}
         super().__init__(f"{names.get(status, status)}: {message}")
 
 

@@ -344,11 +344,22 @@ pa_status pa_reserve_slots(pa_pool *p, const int32_t *seq_ids, const int32_t *nt
     if (total > 0 && !slot_mapping_out) return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: null slot_mapping_out");
 
     const int32_t B = p->cfg.block_size;
+    // Blocks the call must open at block boundaries (copies on write need more): a
+    // request that cannot fit fails here, before anything is allocated, so a huge
+    // count costs nothing and the journal below is sized by what can really happen.
+    int64_t opened = 0;
+    for (int32_t i = 0; i < n; ++i)
+        opened += ((int64_t)seqs[i]->len + ntok[i] + B - 1) / B - (int64_t)seqs[i]->table.size();
+    if (opened > (int64_t)p->free_stack.size() + p->ev_count)
+        return fail(PA_ERR_OUT_OF_BLOCKS, "pa_reserve_slots: no free KV blocks left in the pool (needs " +
+                                              std::to_string(opened) + " new blocks; no change made)");
     std::vector<Undo> journal;
-    journal.reserve((size_t)total + 16);   // one length record per token, more only at block boundaries
     int32_t cows = 0;
     int64_t k = 0;
     pa_status st = PA_OK;
+    try {
+    // one length record per token and two per opened block; a copy on write adds four
+    journal.reserve((size_t)(total + 2 * opened + 16));
     for (int32_t i = 0; i < n && st == PA_OK; ++i) {
         pa_pool::Seq &s = *seqs[i];
         for (int32_t t = 0; t < ntok[i]; ++t) {
@@ -386,6 +397,9 @@ pa_status pa_reserve_slots(pa_pool *p, const int32_t *seq_ids, const int32_t *nt
             s.len = L + 1;
             journal.push_back({Undo::kLen, seq_ids[i], L, 0, 0});
         }
+    }
+    } catch (const std::bad_alloc &) {   // host memory for the journal or a table: undo, report
+        st = fail(PA_ERR_HOST_MEMORY, "host memory allocation failed");
     }
     if (st != PA_OK) {
         std::string msg = pa_last_error();

@@ -285,3 +285,25 @@ def test_duplicate_ids_rejected_without_change_and_next_call_unaffected():
     ta, tb = pa.pa_seq_info(p, a)[1], pa.pa_seq_info(p, b)[1]
     assert slots.tolist() == [int(tb[0]) * 16 + 5, int(ta[0]) * 16 + 3]
     pa.pa_pool_destroy(p)
+
+
+def test_counts_far_beyond_the_pool_fail_cleanly():
+    """Counts near INT32_MAX on many sequences are refused as out of blocks before any
+    block is taken (no host memory is sized by them), and the pool is unchanged."""
+    p = pa.pa_pool_create(1, 64, 16, 1, 64, "f16")
+    seqs = [pa.pa_seq_add(p) for _ in range(8)]
+    pa.pa_reserve_slots(p, seqs, [5] * 8)
+    before = (pa.pa_free_list(p).tolist(), [pa.pa_seq_info(p, s)[0] for s in seqs], pa.pa_pool_stats(p))
+    huge = 2**31 - 1 - 5
+    # the refusal comes before any slot is written, so a small output buffer is enough
+    slot_out = np.empty(1024, np.int64)
+    for ntok in ([huge] * 8, [1] * 7 + [huge], [56 * 16 + 12] + [0] * 7):
+        with pytest.raises(pa.PaError) as e:
+            pa.pa_reserve_slots(p, seqs, ntok, slot_out=slot_out)
+        assert e.value.status == pa.PA_ERR_OUT_OF_BLOCKS and "no change made" in str(e.value)
+        assert (pa.pa_free_list(p).tolist(), [pa.pa_seq_info(p, s)[0] for s in seqs],
+                pa.pa_pool_stats(p)) == before
+    # exactly what is left still fits: 56 free blocks, 11 more tokens fill each tail
+    slots, _ = pa.pa_reserve_slots(p, seqs, [56 * 16 + 11] + [11] * 7)
+    assert len(slots) == 56 * 16 + 11 * 8 and pa.pa_num_free_blocks(p) == 0
+    pa.pa_pool_destroy(p)
