@@ -58,6 +58,9 @@ def parse(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None, help="timed steps (default 64; 8 for large_pool)")
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--repeats", type=int, default=None,
+                    help="timed passes of --steps steps each, over a longer schedule; the median pass is "
+                         "reported (default 7; 3 for large_pool)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="continuous_batch", choices=WORKLOADS)
     ap.add_argument("--split", type=int, default=None, help="tokens per split-K range (0: never split)")
@@ -77,6 +80,9 @@ def parse(argv=None):
         a.steps = 8 if a.workload.startswith("large_pool") or a.workload in ("swap", "prefill") else 64
     if a.split is None:
         a.split = default_split(a.workload)
+    if a.repeats is None:
+        a.repeats = 3 if a.workload.startswith("large_pool") else 7
+    a.repeats = max(1, a.repeats)
     if a.kv_dtype == "fp8" and a.workload not in ("continuous_batch", "large_pool_b16", "large_pool_b32",
                                                     "worked_example"):
         ap.error("--kv-dtype fp8 runs the continuous_batch, large_pool and worked_example workloads")
@@ -84,21 +90,19 @@ def parse(argv=None):
 
 
 def captured_traffic(fp8=False):
-    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if the
-    kernel sources are still the ones that were captured (else None)."""
+    """DRAM bytes per launch of the decode kernel from profiles/traffic.json (one ncu
+    capture), if every kernel source it lists still has the hash it was captured at
+    (else None)."""
     import hashlib
-    import re
-    name = "decode_fp8_continuous_batch.md" if fp8 else "decode_mma_continuous_batch.md"
     csrc = os.path.join(ROOT, "paged_kv_cache_403_b200", "csrc")
     try:
-        text = open(os.path.join(ROOT, "profiles", name)).read()
-        gb = float(re.search(r"traffic per launch \(read \+ write\) \| ([0-9.]+) GB", text).group(1))
-        for src, sha in re.findall(r"([a-z0-9_]+\.cuh?) sha256 prefix at capture: ([0-9a-f]+)", text):
+        entry = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["decode_fp8" if fp8 else "decode_bf16"]
+        for src, sha in entry["sources"].items():
             if not hashlib.sha256(open(os.path.join(csrc, src), "rb").read()).hexdigest().startswith(sha):
                 return None
-    except (OSError, AttributeError):
+        return int(entry["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError, TypeError):
         return None
-    return int(gb * 1e9)
 
 
 # ---------------------------------------------------------------------------- schedules
@@ -164,6 +168,19 @@ def describe(workload):
                          "with one 1024-token system prompt, block 16, 32 q / 8 KV heads, d128, bf16, "
                          "p_stop 1/200, 1 layer",
     }[workload]
+
+
+def arm_config(args, sh, n, world):
+    """The JSON line's config: the workload and its sizes (the same dict on both arms)."""
+    fp8 = args.kv_dtype == "fp8"
+    return {"workload": describe(args.workload), "n_seqs": n, "num_layers": sh.num_layers,
+            "block_size": sh.block_size, "num_q_heads": sh.num_q_heads, "num_kv_heads": sh.num_kv_heads,
+            "head_dim": sh.head_dim, "split_tokens": args.split, "parallelism": f"replicas x{world}",
+            "kv_cache": "E4M3 codes + one power-of-two scale byte per (token, KV head) row" if fp8 else sh.dtype,
+            "l2": (f"flushed: every step first writes {FLUSH_BYTES >> 20} MiB on the compute stream "
+                   "(inside the step time, outside the attention events)"
+                   if args.workload in L2_RESIDENT else
+                   "no flush: the KV read per step exceeds the 126 MB L2")}
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -534,11 +551,12 @@ def run_ours(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
 
-    K, W = args.steps, args.warmup
+    K, W, R = args.steps, args.warmup, args.repeats
     e2e = not args.no_e2e
-    total = W + K + (K if e2e else 0)
+    RE = min(R, 3) if e2e else 0          # end-to-end passes
+    total = W + R * K + RE * K
     recipe = make_recipe(args.workload, replica_seed(rank), total)
-    rep = Replica(torch, args.workload, recipe, total, args.split, device, W + K if e2e else None,
+    rep = Replica(torch, args.workload, recipe, total, args.split, device, W + R * K if e2e else None,
                   prefix_cache=args.prefix_cache == "on", kv_fp8=args.kv_dtype == "fp8")
 
     def barrier():
@@ -556,46 +574,63 @@ def run_ours(args):
     clocks = ClockSampler(local)
     clocks.start()
     lc0 = pa.pa_launch_count()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record(rep.compute)
-    for t in range(W, W + K):
-        rep.step(t)
-    ev1.record(rep.compute)
-    barrier()
-    launches = pa.pa_launch_count() - lc0
-    ms = ev0.elapsed_time(ev1)
-    kv_bytes = sum(rep.kv_bytes)
-    prompt_rows = sum(rep.prompt_rows_appended)
+    # R passes of K steps each over one continuing schedule; every pass is bracketed by a
+    # barrier and a device synchronisation, and the median pass is reported
+    pass_ms, pass_kv = [], []
+    for r in range(R):
+        barrier()
+        kv0 = len(rep.kv_bytes)
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(rep.compute)
+        for t in range(W + r * K, W + (r + 1) * K):
+            rep.step(t)
+        ev1.record(rep.compute)
+        barrier()
+        pass_ms.append(ev0.elapsed_time(ev1))
+        pass_kv.append(sum(rep.kv_bytes[kv0:]))
+    launches = (pa.pa_launch_count() - lc0) / R
+    prompt_rows = sum(rep.prompt_rows_appended) / R
     attn_ms = [a.elapsed_time(b) for a, b in rep.attn_events]
-    alg_per_launch = sum(rep.alg_bytes) / (K * rep.NL)
-    host_ms = 1e3 * sum(rep.host_s) / K
+    alg_per_launch = sum(rep.alg_bytes) / (R * K * rep.NL)
+    host_ms = 1e3 * sum(rep.host_s) / (R * K)
 
-    e2e_ms = e2e_kv = 0.0
+    e2e_ms, e2e_kv = [], []
     e2e_io = (0, 0)
     if e2e:
-        rep.kv_bytes.clear()
         rep.host_s.clear()
         rep.h2d.clear()
         rep.d2h.clear()
-        barrier()
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(rep.compute)
-        for t in range(W + K, W + 2 * K):
-            rep.step(t, e2e=True, time_attention=False)
-        rep.drain()
-        t1.record(rep.compute)
-        barrier()
-        e2e_ms, e2e_kv = t0.elapsed_time(t1), sum(rep.kv_bytes)
-        e2e_host_ms = 1e3 * sum(rep.host_s) / K
-        e2e_io = (sum(rep.h2d) / K, sum(rep.d2h) / K)
+        for r in range(RE):
+            barrier()
+            kv0 = len(rep.kv_bytes)
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record(rep.compute)
+            base = W + R * K + r * K
+            for t in range(base, base + K):
+                rep.step(t, e2e=True, time_attention=False)
+            rep.drain()
+            t1.record(rep.compute)
+            barrier()
+            e2e_ms.append(t0.elapsed_time(t1))
+            e2e_kv.append(sum(rep.kv_bytes[kv0:]))
+        e2e_host_ms = 1e3 * sum(rep.host_s) / (RE * K)
+        e2e_io = (sum(rep.h2d) / (RE * K), sum(rep.d2h) / (RE * K))
     clk = clocks.stop()
 
-    if world > 1:
-        (ms, e2e_ms), (kv_tot, e2e_kv) = combine_ranks(dist, [ms, e2e_ms], [kv_bytes, e2e_kv], device)
-    else:
-        kv_tot = kv_bytes
+    if world > 1:   # per pass: the slowest rank's time, every rank's bytes
+        times, byts = combine_ranks(dist, pass_ms + e2e_ms, pass_kv + e2e_kv, device)
+        pass_ms, e2e_ms = times[:R], times[R:]
+        pass_kv, e2e_kv = byts[:R], byts[R:]
+
+    def median_pass(ms_list, kv_list):
+        i = int(np.argsort(ms_list)[len(ms_list) // 2])
+        return ms_list[i], kv_list[i]
+
+    ms, kv_tot = median_pass(pass_ms, pass_kv)
+    if e2e:
+        e2e_ms_med, e2e_kv_med = median_pass(e2e_ms, e2e_kv)
 
     if rank == 0:
         peaks = {}
@@ -613,16 +648,9 @@ def run_ours(args):
             "warmup": W, "ms_per_step": round(ms / K, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp8_e4m3 cache, " + sh.dtype if rep.kv_fp8 else sh.dtype,
             "data": "synthetic (seeded counter-based K/V/q values; seeded lengths, pool order and stops)",
-            "config": {"workload": describe(args.workload), "n_seqs": rep.n, "num_layers": rep.NL,
-                       "block_size": sh.block_size, "num_q_heads": sh.num_q_heads,
-                       "num_kv_heads": sh.num_kv_heads, "head_dim": sh.head_dim, "split_tokens": args.split,
-                       "parallelism": f"replicas x{world}",
-                       "kv_cache": ("E4M3 codes + one power-of-two scale byte per (token, KV head) row"
-                                    if rep.kv_fp8 else sh.dtype),
-                       "l2": (f"flushed: every step first writes {FLUSH_BYTES >> 20} MiB on the compute stream "
-                              "(inside the step time, outside the attention events)"
-                              if rep.flush is not None else
-                              "no flush: the KV read per step exceeds the 126 MB L2")},
+            "config": arm_config(args, sh, rep.n, world),
+            "passes": {"n": R, "ms_per_step": [round(x / K, 4) for x in pass_ms],
+                       "reported": "median pass; each pass is --steps steps of one continuing schedule"},
             "decode_tokens_per_s": round(world * rep.n * K / (ms * 1e-3), 1),
             "kv_gb_per_step": round(kv_tot / K / 1e9 / world, 4),
             "hbm_fraction_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
@@ -648,9 +676,10 @@ def run_ours(args):
         if args.workload == "shared_prompt":
             line["config"]["prefix_cache"] = args.prefix_cache
         if e2e:
-            line["e2e"] = {"value": round(e2e_kv / (e2e_ms * 1e-3) / 1e9, 1), "unit": UNIT,
+            line["e2e"] = {"value": round(e2e_kv_med / (e2e_ms_med * 1e-3) / 1e9, 1), "unit": UNIT,
                            "h2d_bytes_per_step": int(e2e_io[0]), "d2h_bytes_per_step": int(e2e_io[1]),
-                           "ms_per_step": round(e2e_ms / K, 4), "host_ms_per_step": round(e2e_host_ms, 4)}
+                           "ms_per_step": round(e2e_ms_med / K, 4), "host_ms_per_step": round(e2e_host_ms, 4),
+                           "passes": {"n": RE, "ms_per_step": [round(x / K, 4) for x in e2e_ms]}}
         if not args.no_cpu_baseline and args.workload not in ("prefix_sharing", "shared_prompt") and not rep.kv_fp8:
             line["cpu_baseline"] = cpu_baseline(rep, args.cpu_sample_seqs, W, args.cpu_seconds)
         print(json.dumps(line), flush=True)
@@ -735,6 +764,8 @@ def run_reference(args):
         return
     import oracle
     from synthetic import workloads as wl
+    if args.workload != "continuous_batch" or args.kv_dtype != "native":
+        raise SystemExit("bench.py --impl reference times the oracle on the continuous batch (bf16 cache) only")
     K, W = args.steps, args.warmup
     recipe = wl.continuous_batch(seed=3, steps=W + K)
     plan = simulate(recipe["schedule"], len(recipe["schedule"].initial), W + K)
@@ -752,7 +783,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": round(dt_tot / K * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": describe("continuous_batch"), "parallelism": "cpu"},
+            "config": arm_config(args, recipe["shape"], len(recipe["schedule"].initial), world),
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oracle.max_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

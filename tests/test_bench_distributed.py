@@ -39,8 +39,9 @@ def test_two_gloo_ranks_combine_time_max_and_bytes_sum():
     assert out[0][2] != out[1][2]             # each replica draws its own workload
 
 
-class _Args:
-    steps, warmup = 1, 0
+def _Args():
+    import bench
+    return bench.parse(["--impl", "reference", "--steps", "1", "--warmup", "0"])
 
 
 def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
@@ -63,3 +64,7 @@ def test_reference_arm_prints_one_json_line(monkeypatch, capsys):
     assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "GB/s"
     assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    # the same config dict the GPU arm prints for the same command line
+    from synthetic import workloads as wl
+    r = wl.continuous_batch()
+    assert d["config"] == bench.arm_config(_Args(), r["shape"], len(r["schedule"].initial), 1)
