@@ -20,10 +20,11 @@
 //                    only when a score passes the running maximum by 2^8), P written
 //                    back to TMEM (tcgen05.st) as the A operand of P V: for bf16 a
 //                    truncated high part plus the rounded remainder, for fp16 once;
-//   warp 8           tensor-core issue (one lane): S_t = Q_t K^T (M=128, N=64, both
-//                    operands in shared memory) and O_t += P_t V (M=128, N=head_dim,
-//                    per part of P; A = P from TMEM, B = V from shared memory);
-//   warp 9           TMA producer: 128-key tiles of K and V (2-D tensor loads, 128-byte
+//   warp 16          tensor-core issue (one lane): S_t = Q_t K^T (M=128, N=128 keys,
+//                    both operands in shared memory) and O_t += P_t V (M=128,
+//                    N=head_dim, per part of P; A = P from TMEM, B = V from shared
+//                    memory);
+//   warp 17          TMA producer: 128-key tiles of K and V (2-D tensor loads, 128-byte
 //                    swizzle) into a 2-stage ring, walking the block table.
 // Tiles of 128 keys make S = Q K^T an M=128, N=128 product: at N=64 the tensor core ran
 // it at about a third of its rate.  TMEM then holds O and S of both query tiles (512
