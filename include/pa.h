@@ -317,6 +317,8 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
  *    PA_ERR_INVALID_ARG and a message naming both sizes; nothing is launched.
  *  - The first call on a device looks up the array's device address with that
  *    device current and keeps it; make that first call before any stream capture.
+ *    The kept address belongs to the device's context: after cudaDeviceReset the
+ *    entry must not be called again in the same process.
  *  - All calls on a device share the one array and it keeps the last call's
  *    contents.  Nothing in it needs to start at zero (every partial a call reads
  *    was written earlier in the same call), but calls that overlap on the GPU --
@@ -355,6 +357,19 @@ pa_status pa_prefill_attention(pa_pool *pool, int32_t layer, const void *q, void
 pa_status pa_device_error(int32_t *code, int32_t clear);
 /* Kernels this library has launched since it was loaded (all devices). */
 uint64_t pa_launch_count(void);
+
+/* Failure-detection test hook (no page counterpart; the pages' failure cases --
+ * [P3] "Decisions leaders and practitioners actually face": reject cleanly rather
+ * than stall -- only motivate it).  Every device-side wait of the library's kernels
+ * is bounded; this sets the bound on the current device to wait_limit_ns
+ * (<= 0 restores the default of 2 s) and, when withhold_cta >= 0, makes the
+ * producer warp of the decode CTA with that linear block index issue no copies
+ * (every later pa_decode_attention launch on any device, until called again with
+ * -1).  That CTA's consumers then wait for data that never comes: each wait runs
+ * out after the bound, records device error bit 4 and returns, no copy is left in
+ * flight, and the rest of the launch is unaffected; the withheld CTA's outputs are
+ * not meaningful.  Off by default; synchronises the device. */
+pa_status pa_debug_wait_test(int64_t wait_limit_ns, int32_t withhold_cta);
 
 #ifdef __cplusplus
 }

@@ -314,6 +314,12 @@ def pa_device_error(clear: bool = False) -> int:
     return code.value
 
 
+def pa_debug_wait_test(wait_limit_ns: int = 0, withhold_cta: int = -1) -> None:
+    """Failure-detection test hook: bound of every device-side wait (0: the 2 s
+    default) and the decode CTA whose copies are withheld (-1: none)."""
+    _check(_lib().pa_debug_wait_test(int(wait_limit_ns), int(withhold_cta)))
+
+
 def pa_launch_count() -> int:
     return int(_lib().pa_launch_count())
 

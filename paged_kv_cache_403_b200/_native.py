@@ -64,6 +64,7 @@ SIGNATURES = {
     "pa_prefill_attention": (ctypes.c_int, [c_vp, c_i32, c_vp, c_vp, ctypes.c_int, c_vp, c_i32, c_vp, c_vp,
                                             c_i32, c_i32, c_i32, c_f32, c_vp]),
     "pa_device_error": (ctypes.c_int, [P_i32, c_i32]),
+    "pa_debug_wait_test": (ctypes.c_int, [c_i64, c_i32]),
     "pa_launch_count": (c_u64, []),
 }
 

@@ -297,6 +297,7 @@ pa_status pa_seq_fork(pa_pool *p, int32_t parent, int32_t *child) {
 }
 
 pa_status pa_seq_free(pa_pool *p, int32_t seq_id) {
+    pa_internal::TraceRange trace_("pa_seq_free");
     if (!p) return fail(PA_ERR_INVALID_ARG, "pa_seq_free: null pool");
     auto it = p->seqs.find(seq_id);
     if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_seq_free: unknown sequence");
@@ -324,6 +325,7 @@ pa_status pa_seq_info(const pa_pool *p, int32_t seq_id, int32_t *len, int32_t *t
 
 pa_status pa_reserve_slots(pa_pool *p, const int32_t *seq_ids, const int32_t *ntok, int32_t n,
                            int64_t *slot_mapping_out, int32_t *cow_pairs_out, int32_t *n_cow) {
+    pa_internal::TraceRange trace_("pa_reserve_slots");
     if (!p || n < 0 || (n > 0 && (!seq_ids || !ntok)))
         return fail(PA_ERR_INVALID_ARG, "pa_reserve_slots: bad argument");
     int64_t total = 0;
@@ -434,6 +436,7 @@ pa_status pa_reserve_slots(pa_pool *p, const int32_t *seq_ids, const int32_t *nt
 
 pa_status pa_build_block_tables(const pa_pool *p, const int32_t *seq_ids, int32_t n, int32_t max_blocks,
                                 int32_t *tables_out, int32_t *lens_out) {
+    pa_internal::TraceRange trace_("pa_build_block_tables");
     if (!p || n < 0 || max_blocks < 1 || (n > 0 && (!seq_ids || !tables_out || !lens_out)))
         return fail(PA_ERR_INVALID_ARG, "pa_build_block_tables: bad argument");
     for (int32_t i = 0; i < n; ++i) {
@@ -519,6 +522,7 @@ pa_status pa_swap_bytes(const pa_pool *p, int32_t seq_id, size_t *bytes) {
 }
 
 pa_status pa_swap_out(pa_pool *p, int32_t seq_id, void *host_buf, size_t buf_bytes, pa_stream stream) {
+    pa_internal::TraceRange trace_("pa_swap_out");
     if (!p) return fail(PA_ERR_INVALID_ARG, "pa_swap_out: null pool");
     auto it = p->seqs.find(seq_id);
     if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_swap_out: unknown sequence");
@@ -538,6 +542,7 @@ pa_status pa_swap_out(pa_pool *p, int32_t seq_id, void *host_buf, size_t buf_byt
 }
 
 pa_status pa_swap_in(pa_pool *p, int32_t seq_id, const void *host_buf, size_t buf_bytes, pa_stream stream) {
+    pa_internal::TraceRange trace_("pa_swap_in");
     if (!p) return fail(PA_ERR_INVALID_ARG, "pa_swap_in: null pool");
     auto it = p->seqs.find(seq_id);
     if (it == p->seqs.end()) return fail(PA_ERR_INVALID_ARG, "pa_swap_in: unknown sequence");

@@ -154,6 +154,7 @@ struct Params {
     int32_t *counters;              // [n_seqs][head_groups] split-merge counters
     int32_t max_blocks, num_blocks, num_kv_heads, num_q_heads, layer;
     int32_t split_blocks, max_splits, out_f32, group, head_groups;
+    int32_t debug_withhold;         // see copies_withheld(); -1 outside wait-expiry tests
     float scale_log2;
 };
 
@@ -251,7 +252,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const __grid_
         const int32_t *trow = p.tables + (size_t)s * p.max_blocks + b0;
         bool ok = true;
         int issued = 0;
-        for (int base = 0; base < ntiles && ok; base += 32) {
+        const int to_issue = copies_withheld(p.debug_withhold) ? 0 : ntiles;
+        for (int base = 0; base < to_issue && ok; base += 32) {
             int blk = 0;
             if (base + lane < ntiles) {
                 blk = trow[base + lane];

@@ -33,9 +33,11 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <string>
+#include <type_traits>
 
 #include "pool.hpp"
 
@@ -89,15 +91,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
-// Waits are bounded: after kWaitLimitNs the waiter records kErrTimeout and gives up.
+// Waits are bounded: after g_wait_limit_ns (kWaitLimitNs unless a test lowers it
+// through pa_debug_wait_test) the waiter records kErrTimeout and gives up.  The bound
+// is read only once a wait has to spin, so the common path never loads it.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+
+__device__ __forceinline__ uint64_t wait_limit_ns() { return *static_cast<volatile uint64_t *>(&g_wait_limit_ns); }
+
+// A wait-expiry test (pa_debug_wait_test) names one decode CTA, by its linear block
+// index, whose producer issues no copies, so that its consumers' waits run out.
+__device__ __forceinline__ bool copies_withheld(int32_t withhold) {
+    return withhold >= 0 &&
+           (int64_t)blockIdx.x + (int64_t)gridDim.x * (blockIdx.y + (int64_t)gridDim.y * blockIdx.z) == withhold;
+}
 
 // One thread waits (the producer lane).
 __device__ __forceinline__ bool mbar_wait_thread(uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
+    const uint64_t t0 = global_timer_ns(), limit = wait_limit_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit) {
             raise_error(kErrTimeout);
             return false;
         }
@@ -117,12 +131,15 @@ __device__ __forceinline__ void drain_copies(uint64_t *full, int issued, int sta
 
 // A whole warp waits and leaves together, so later full-warp shuffles stay converged.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity) {
-    uint64_t t0 = 0;
+    uint64_t t0 = 0, limit = kWaitLimitNs;
     for (uint32_t it = 0;; ++it) {
         const bool done = mbar_try_wait(bar, parity);
         if (__all_sync(0xffffffffu, done)) return true;
-        if (it == 0) t0 = global_timer_ns();
-        const bool late = global_timer_ns() - t0 > kWaitLimitNs;
+        if (it == 0) {
+            t0 = global_timer_ns();
+            limit = wait_limit_ns();
+        }
+        const bool late = global_timer_ns() - t0 > limit;
         if (__any_sync(0xffffffffu, late)) {
             if ((threadIdx.x & 31) == 0) raise_error(kErrTimeout);
             return false;
@@ -241,6 +258,7 @@ struct DecodeParams {
     float *ws_ml;                   // [n][max_splits][Hq][2]
     int32_t n_seqs, max_blocks, num_blocks, num_kv_heads, num_q_heads;
     int32_t split_blocks, max_splits, out_f32;
+    int32_t debug_withhold;         // see copies_withheld(); -1 outside wait-expiry tests
     float scale_log2;
 };
 
@@ -332,7 +350,8 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_simt_kernel(const
         const int32_t *trow = p.tables + (size_t)s * p.max_blocks + b0;
         bool ok = true;
         int issued = 0;
-        for (int base = 0; base < ntiles && ok; base += 32) {
+        const int to_issue = copies_withheld(p.debug_withhold) ? 0 : ntiles;
+        for (int base = 0; base < to_issue && ok; base += 32) {
             int blk = 0;
             if (base + lane < ntiles) {
                 blk = trow[base + lane];
@@ -835,6 +854,7 @@ struct MmaParams {
     int32_t *counters;              // [n_seqs][head_groups] split-merge counters
     int32_t max_blocks, num_blocks, num_kv_heads, num_q_heads, layer;
     int32_t split_blocks, max_splits, out_f32, heads_per_cta, head_groups;
+    int32_t debug_withhold;         // see copies_withheld(); -1 outside wait-expiry tests
     float scale_log2;
 };
 
@@ -921,7 +941,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) paged_decode_mma_kernel(con
         const int32_t *trow = p.tables + (size_t)s * p.max_blocks + b0;
         bool ok = true;
         int issued = 0;
-        for (int base = 0; base < ntiles && ok; base += 32) {
+        const int to_issue = copies_withheld(p.debug_withhold) ? 0 : ntiles;
+        for (int base = 0; base < to_issue && ok; base += 32) {
             int blk = 0;
             if (base + lane < ntiles) {
                 blk = trow[base + lane];
@@ -1383,6 +1404,9 @@ pa_status launch_prefill(const prefill::Params &p, dim3 grid, cudaStream_t strea
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Decode CTA whose copies a wait-expiry test withholds (pa_debug_wait_test), else -1.
+std::atomic<int32_t> g_debug_withhold{-1};
+
 // Decode workspace: split partials (acc [parts][D] then (m, l) [parts][2], fp32) when a
 // sequence can have more than one split, then the longest-first range order
 // (int32 [n_seqs * max_splits]), each part rounded up to 16 bytes.
@@ -1415,21 +1439,23 @@ namespace {
 // Device address of the scratch array on the current device.  Host code cannot pass
 // the array's name to a kernel (on the host it is only a stand-in symbol), so the
 // first call on each device looks the address up with that device current and
-// keeps it.
+// keeps it.  Host threads may make their first calls at the same time: each looks
+// the address up (the same value) and publishes it atomically.  The kept address
+// belongs to the device's current context; after cudaDeviceReset it is stale.
 pa_status static_scratch_address(void **out) {
-    static void *addr[64] = {};
+    static std::atomic<void *> addr[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
     if (dev < 0 || dev >= 64) return fail(PA_ERR_UNSUPPORTED, "pa_decode_attention_static: device ordinal >= 64");
-    if (!addr[dev]) {
-        void *p = nullptr;
+    void *p = addr[dev].load(std::memory_order_acquire);
+    if (!p) {
         e = cudaGetSymbolAddress(&p, pa_static_split_scratch);
         if (e != cudaSuccess || !p)
             return fail(PA_ERR_CUDA, std::string("cudaGetSymbolAddress(split scratch): ") + cudaGetErrorString(e));
-        addr[dev] = p;
+        addr[dev].store(p, std::memory_order_release);
     }
-    *out = addr[dev];
+    *out = p;
     return PA_OK;
 }
 
@@ -1455,6 +1481,7 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
                               const int32_t *block_tables_dev, int32_t max_blocks, const int32_t *seq_lens_dev,
                               int32_t n_seqs, int32_t num_q_heads, float scale, int32_t split_tokens,
                               void *workspace, size_t ws_bytes, pa_stream stream) {
+    pa_internal::TraceRange trace_("pa_decode_attention");
     if (!pool || !pool->device_ready())
         return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: pool has no device memory (or no FP8 scales)");
     const pa_pool_config &c = pool->cfg;
@@ -1562,6 +1589,7 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
         p.max_splits = max_splits;
         p.out_f32 = r.out_f32;
         p.scale_log2 = scale_log2;
+        p.debug_withhold = g_debug_withhold.load(std::memory_order_relaxed);
         const int hpc = group < 4 ? group : 4;
         return dispatch_simt<float>(p, r, c.block_size, c.head_dim, hpc, st);
     }
@@ -1592,6 +1620,7 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
         p.order = order;
         p.counters = counters;
         p.scale_log2 = scale_log2;
+        p.debug_withhold = g_debug_withhold.load(std::memory_order_relaxed);
         const bool bf = c.act_dtype == PA_BF16;
 #define PA_FP8_LAUNCH(B, H) \
     (bf ? launch_fp8<__nv_bfloat16, B, H>(p, r, n_seqs, st) : launch_fp8<__half, B, H>(p, r, n_seqs, st))
@@ -1631,6 +1660,7 @@ pa_status pa_decode_attention(pa_pool *pool, int32_t layer, const void *q, void 
     p.order = order;
     p.counters = counters;
     p.scale_log2 = scale_log2;
+    p.debug_withhold = g_debug_withhold.load(std::memory_order_relaxed);
     if (c.dtype == PA_BF16) return dispatch_mma<__nv_bfloat16>(p, r, n_seqs, c.block_size, c.head_dim, st);
     return dispatch_mma<__half>(p, r, n_seqs, c.block_size, c.head_dim, st);
 }
@@ -1639,6 +1669,7 @@ pa_status pa_prefill_attention(pa_pool *pool, int32_t layer, const void *q, void
                                const int32_t *block_tables_dev, int32_t max_blocks, const int32_t *seq_lens_dev,
                                const int32_t *q_start_dev, int32_t n_seqs, int32_t max_q_len, int32_t num_q_heads,
                                float scale, pa_stream stream) {
+    pa_internal::TraceRange trace_("pa_prefill_attention");
     if (!pool || !pool->k_pool) return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: pool has no device memory");
     const pa_pool_config &c = pool->cfg;
     if (layer < 0 || layer >= c.num_layers) return fail(PA_ERR_INVALID_ARG, "pa_prefill_attention: layer out of range");
@@ -1694,6 +1725,7 @@ pa_status pa_prefill_attention(pa_pool *pool, int32_t layer, const void *q, void
 
 pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const void *v_new,
                        const int64_t *slot_mapping_dev, int32_t n_tokens, pa_stream stream) {
+    pa_internal::TraceRange trace_("pa_append_kv");
     if (!pool || !pool->device_ready())
         return fail(PA_ERR_INVALID_ARG, "pa_append_kv: pool has no device memory (or no FP8 scales)");
     if (layer < 0 || layer >= pool->cfg.num_layers) return fail(PA_ERR_INVALID_ARG, "pa_append_kv: layer out of range");
@@ -1755,6 +1787,7 @@ pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const vo
 }
 
 pa_status pa_copy_blocks(pa_pool *pool, const int32_t *pairs_dev, int32_t n_pairs, pa_stream stream) {
+    pa_internal::TraceRange trace_("pa_copy_blocks");
     if (!pool || !pool->device_ready())
         return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: pool has no device memory (or no FP8 scales)");
     if (n_pairs < 0) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: negative n_pairs");
@@ -1781,6 +1814,7 @@ pa_status pa_decode_attention_static(pa_pool *pool, int32_t layer, const void *q
                                      const int32_t *block_tables_dev, int32_t max_blocks, const int32_t *seq_lens_dev,
                                      int32_t n_seqs, int32_t num_q_heads, float scale, int32_t split_tokens,
                                      pa_stream stream) {
+    pa_internal::TraceRange trace_("pa_decode_attention_static");
     if (!pool) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention_static: null pool");
     if (n_seqs < 0 || max_blocks < 1 || split_tokens < 0)
         return fail(PA_ERR_INVALID_ARG, "pa_decode_attention_static: bad n_seqs, max_blocks or split_tokens");
@@ -1803,6 +1837,17 @@ pa_status pa_decode_attention_static(pa_pool *pool, int32_t layer, const void *q
     return pa_decode_attention(pool, layer, q, out, out_dtype, block_tables_dev, max_blocks, seq_lens_dev, n_seqs,
                                num_q_heads, scale, split_tokens, ws, need > 0 ? (size_t)PA_STATIC_WORKSPACE_BYTES : 0,
                                stream);
+}
+
+pa_status pa_debug_wait_test(int64_t wait_limit_ns, int32_t withhold_cta) {
+    if (withhold_cta < -1) return fail(PA_ERR_INVALID_ARG, "pa_debug_wait_test: withhold_cta must be >= -1");
+    const uint64_t limit = wait_limit_ns > 0 ? (uint64_t)wait_limit_ns : kWaitLimitNs;
+    cudaError_t e = cudaDeviceSynchronize();   // no launch in flight sees a half-changed setting
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_wait_limit_ns, &limit, sizeof limit);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, std::string("pa_debug_wait_test: ") + cudaGetErrorString(e));
+    g_debug_withhold.store(withhold_cta, std::memory_order_relaxed);
+    return PA_OK;
 }
 
 pa_status pa_device_error(int32_t *code, int32_t clear) {

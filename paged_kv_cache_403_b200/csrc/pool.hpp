@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <cstdint>
@@ -74,6 +75,16 @@ struct pa_pool {
 };
 
 namespace pa_internal {
+// NVTX range named after a library call, so profiler timelines (Nsight Systems, the
+// NVTX filters of Nsight Compute) show where each call's host work and launches sit.
+// Without a tool attached a push or pop is a check of one function pointer.
+struct TraceRange {
+    explicit TraceRange(const char *name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+    TraceRange(const TraceRange &) = delete;
+    TraceRange &operator=(const TraceRange &) = delete;
+};
+
 // Records `msg` as this thread's last error and returns `st`.
 pa_status fail(pa_status st, const std::string &msg);
 pa_status ok();

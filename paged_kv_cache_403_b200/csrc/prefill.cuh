@@ -143,14 +143,17 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Bounded wait for a whole warp (lanes leave together); gives up when another role has
-// set the abort flag or after kWaitLimitNs, setting the flag itself then.
+// set the abort flag or after the wait bound (wait_limit_ns()), setting the flag itself then.
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-    uint64_t t0 = 0;
+    uint64_t t0 = 0, limit = kWaitLimitNs;
     for (uint32_t it = 0;; ++it) {
         const bool done = mbar_try_wait(bar, parity);
         if (__all_sync(0xffffffffu, done)) return true;
-        if (it == 0) t0 = global_timer_ns();
-        const bool give_up = *abort_flag || global_timer_ns() - t0 > kWaitLimitNs;
+        if (it == 0) {
+            t0 = global_timer_ns();
+            limit = wait_limit_ns();
+        }
+        const bool give_up = *abort_flag || global_timer_ns() - t0 > limit;
         if (__any_sync(0xffffffffu, give_up)) {
             if ((threadIdx.x & 31) == 0 && !*abort_flag) {
                 raise_error(kErrTimeout);
