@@ -122,3 +122,60 @@ def sequence_attention_fp8(shape, seed, layer, uid, length, q_uid, q_pos):
     q = sv.rows(sv.KIND_Q, seed, layer, [q_uid], [q_pos], shape.num_q_heads, d, shape.q_scale, shape.dtype)
     return oracle.paged_decode_fp8(lay(kc), lay(vc), lay(ks), lay(vs), np.arange(nblk, dtype=np.int32)[None],
                                    np.array([length]), q, shape.dtype, 1.0 / math.sqrt(d))[0]
+
+
+STORAGE = {"f32": np.float32, "f16": np.float16, "bf16": np.uint16}
+
+
+def histories_attention(shape, seed, layer, uids, lens, q_positions, rows=None):
+    """fp64 attention of every sequence of a batch against its whole regenerated history
+    (position p of sequence i written by uid uids[i] as token p), in one oracle call.
+
+    rows(kind, uids, toks) -> host storage rows [len][num_kv_heads][head_dim]; by default
+    the host generator.  Each history is laid into its own run of blocks of a contiguous
+    host pool with an identity-like block table, so this checks the GPU's gather through
+    its own shuffled tables against plain contiguous reads.
+    """
+    B, hkv, d = shape.block_size, shape.num_kv_heads, shape.head_dim
+    if rows is None:
+        def rows(kind, u, t):
+            return sv.rows(kind, seed, layer, u, t, hkv, d, shape.kv_scale, shape.dtype)
+    lens = np.asarray(lens, np.int64)
+    nblk = -(-lens // B)
+    first = np.concatenate([[0], np.cumsum(nblk)[:-1]]).astype(np.int64)
+    kp = np.zeros((int(nblk.sum()), hkv, B, d), STORAGE[shape.dtype])
+    vp = np.zeros_like(kp)
+    for i, (uid, L) in enumerate(zip(uids, lens)):
+        L = int(L)
+        toks = np.arange(L)
+        u = np.full(L, int(uid))
+        for kind, pool in ((sv.KIND_K, kp), (sv.KIND_V, vp)):
+            r = np.asarray(rows(kind, u, toks))
+            pad = int(nblk[i]) * B - L
+            if pad:
+                r = np.concatenate([r, np.zeros((pad, hkv, d), r.dtype)])
+            pool[first[i]:first[i] + nblk[i]] = r.reshape(int(nblk[i]), B, hkv, d).transpose(0, 2, 1, 3)
+    tables = np.full((len(lens), int(nblk.max())), -1, np.int32)
+    for i in range(len(lens)):
+        tables[i, :nblk[i]] = first[i] + np.arange(nblk[i])
+    q = sv.rows(sv.KIND_Q, seed, layer, np.asarray(uids), np.asarray(q_positions), shape.num_q_heads, d,
+                shape.q_scale, shape.dtype)
+    return oracle.paged_decode(kp, vp, shape.dtype, tables, lens.astype(np.int32), q, 1.0 / math.sqrt(d))
+
+
+def device_generated_rows(shape, seed, layer):
+    """rows() for histories_attention drawn by the device implementation of the seeded
+    input generator (synthetic/csrc/synth_gen.cu, bit-identical to the host one and
+    tested against it), then copied to the host: the same inputs, made fast enough to
+    regenerate whole full-size batches."""
+    import torch
+    from synthetic import gpu as sgpu
+    dt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[shape.dtype]
+
+    def rows(kind, u, t):
+        out = torch.empty((len(u), shape.num_kv_heads, shape.head_dim), dtype=dt, device="cuda")
+        sgpu.fill_rows(out, kind, seed, layer, torch.from_numpy(np.asarray(u, np.int32)).cuda(),
+                       torch.from_numpy(np.asarray(t, np.int32)).cuda(), shape.kv_scale, shape.dtype)
+        h = out.cpu()
+        return h.view(torch.int16).numpy().view(np.uint16) if dt == torch.bfloat16 else h.numpy()
+    return rows

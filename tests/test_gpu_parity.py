@@ -17,7 +17,7 @@ from paged_kv_cache_403_b200.runners import ContinuousBatch, run_prefix_sharing,
 from synthetic import values as sv
 from synthetic import workloads as wl
 
-from oracle_replay import OracleRun, check_close, sequence_attention
+from oracle_replay import OracleRun, check_close, device_generated_rows, histories_attention, sequence_attention
 
 pytestmark = pytest.mark.gpu
 
@@ -183,14 +183,21 @@ def test_continuous_batch_reduced_full_replay():
 @pytest.mark.parametrize("split", [2048, 4096])
 def test_continuous_batch_full_size_sampled(split):
     """256 sequences, 64 steps, bf16 output, split 4096 as timed by the benchmark (and
-    2048); sampled sequences checked against the oracle on regenerated histories."""
+    2048): sampled sequences of steps 0 and 21, and every sequence of the last step
+    (after retirements and admissions), checked against the oracle on regenerated
+    histories."""
     r = wl.continuous_batch()
     sh = r["shape"]
     cb = ContinuousBatch(r)
     rng = np.random.default_rng(0)
     for t in range(64):
         rec = cb.step(split_tokens=split)
-        if t in (0, 21, 63):
+        if t == 63:
+            ref = histories_attention(sh, r["seed"], 0, rec.uids, rec.lens, rec.positions,
+                                      device_generated_rows(sh, r["seed"], 0))
+            err = check_close(widen(rec.outputs[0]), ref, "bf16", "bf16", f"step {t}, all sequences")
+            print(f"continuous batch split {split}: step 63, all {len(rec.lens)} sequences, max err {err:.3g}")
+        elif t in (0, 21):
             lens = rec.lens
             picks = set(rng.choice(len(lens), size=5, replace=False).tolist())
             picks |= {int(np.argmax(lens)), int(np.argmin(lens))}
@@ -221,12 +228,15 @@ def test_large_pool_sampled(bs, split):
     assert (lens > 4096).any()
     picks = [int(np.argmax(lens)), int(np.argmin(lens)), int(np.argsort(lens)[len(lens) // 2])]
     picks += [int(i) for i in np.nonzero(lens > 4096)[0][:2]]
-    for layer in (0, 31):
-        out = widen(rec.outputs[layer])
-        for i in picks:
-            ref = sequence_attention(sh, r["seed"], layer, rec.uids[i], int(lens[i]), rec.uids[i],
-                                     int(rec.positions[i]))
-            check_close(out[i], ref, "f16", "f16", f"layer {layer} seq {i}")
+    out = widen(rec.outputs[0])
+    for i in picks:
+        ref = sequence_attention(sh, r["seed"], 0, rec.uids[i], int(lens[i]), rec.uids[i], int(rec.positions[i]))
+        check_close(out[i], ref, "f16", "f16", f"layer 0 seq {i}")
+    # every sequence of the last layer
+    ref = histories_attention(sh, r["seed"], 31, rec.uids, lens, rec.positions,
+                              device_generated_rows(sh, r["seed"], 31))
+    err = check_close(widen(rec.outputs[31]), ref, "f16", "f16", "layer 31, all sequences")
+    print(f"large pool B{bs} split {split}: layer 31, all {len(lens)} sequences, max err {err:.3g}")
     del cache
     torch.cuda.empty_cache()
 
