@@ -11,28 +11,29 @@
 // One CTA per (256 query rows, KV head, sequence): two 128-row tiles A and B whose rows
 // are (token, query head of the GQA group) pairs, row = token * G + head, so every
 // query head of the group shares each key/value tile.  Warp roles:
-//   warps 0-15       softmax: warp w serves tile (w / 4) % 2, rows 32 (w % 4) .. +31 (its
-//                    TMEM lane quarter) and keys / O columns 64 (w / 8) .. +63, so two
-//                    threads share a row and exchange their partial maxima (and at the
-//                    end their sums) through shared memory; per row: tcgen05.ld of the
-//                    scores, causal / length mask by select, base-2 online
-//                    softmax with a lazily moved maximum (the O row is rescaled in TMEM
-//                    only when a score passes the running maximum by 2^8), P written
-//                    back to TMEM (tcgen05.st) as the A operand of P V: for bf16 a
-//                    truncated high part plus the rounded remainder, for fp16 once;
-//   warp 16          tensor-core issue (one lane): S_t = Q_t K^T (M=128, N=128 keys,
+//   warps 0-7        softmax, one thread per row: warp w serves tile w / 4 and rows
+//                    32 (w % 4) .. +31 (its TMEM lane quarter), so each SM sub-partition
+//                    holds one softmax warp of each tile.  Per row and key tile: the
+//                    128 scores come out of TMEM in four loads with one wait, the row
+//                    maximum needs no other thread, a causal / length mask by select on
+//                    the last tiles only, base-2 online softmax with a lazily moved
+//                    maximum (the O row is rescaled in TMEM only when a score passes the
+//                    running maximum by 2^8), and P written back to TMEM (tcgen05.st) as
+//                    the A operand of P V: for bf16 a truncated high part plus the
+//                    truncated remainder, for fp16 once;
+//   warp 8           tensor-core issue (one lane): S_t = Q_t K^T (M=128, N=128 keys,
 //                    both operands in shared memory) and O_t += P_t V (M=128,
 //                    N=head_dim, per part of P; A = P from TMEM, B = V from shared
 //                    memory);
-//   warp 17          TMA producer: 128-key tiles of K and V (2-D tensor loads, 128-byte
+//   warp 9           TMA producer: 128-key tiles of K and V (2-D tensor loads, 128-byte
 //                    swizzle) into a 2-stage ring, walking the block table.
 // Tiles of 128 keys make S = Q K^T an M=128, N=128 product: at N=64 the tensor core ran
 // it at about a third of its rate.  TMEM then holds O and S of both query tiles (512
 // columns), so P is written over S in place: the 16 columns of each 16-key group of S
 // take that group's P (8 columns of high parts, 8 of low parts), and the next S of the
 // tile is issued after the P V that reads them (one thread's tcgen05.mma run in order).
-// The two tiles ping-pong: while one warpgroup computes exponentials the tensor core
-// works on the other tile.  Every hand-off is an mbarrier; every wait is bounded and
+// The two tiles ping-pong: while one tile's softmax computes exponentials the tensor
+// core works on the other tile.  Every hand-off is an mbarrier; every wait is bounded and
 // sets a shared abort flag that all roles check; TMEM is always freed.  Key rows past
 // the sequence end are zeroed in shared memory before P V (weight 0, but 0 * NaN would
 // not be 0).
@@ -41,8 +42,7 @@ namespace prefill {
 constexpr int kRows = 128;           // MMA M: rows of one query tile
 constexpr int kTiles = 2;            // query tiles per CTA (ping-pong)
 constexpr int kKeys = 128;           // keys per K/V tile
-constexpr int kHalves = 2;           // softmax threads per row (each: 64 keys, 64 O columns)
-constexpr int kSoftmaxWarps = kTiles * kRows * kHalves / 32;
+constexpr int kSoftmaxWarps = kTiles * kRows / 32;   // one thread per query row
 constexpr int kThreads = kSoftmaxWarps * 32 + 64;   // + tensor-core issue warp + TMA warp
 constexpr int kMmaWarp = kSoftmaxWarps, kTmaWarp = kMmaWarp + 1;
 constexpr int kD = 128;              // head_dim
@@ -54,11 +54,9 @@ constexpr uint32_t kOCol = 0, kSCol = 256;
 constexpr int kQBytes = kRows * kD * 2;         // 32 KB per tile: [2 halves][128 rows][128 B]
 constexpr int kKVBytes = kKeys * kD * 2;        // 32 KB: [2 halves][128 rows][128 B]
 constexpr int kStages = 2;
-// s_full, p_full, o_done per tile; k/v full, empty per stage; one row-exchange barrier
-// per (tile, lane quarter)
-constexpr int kNumBars = 3 * kTiles + 4 * kStages + kTiles * 4;
-constexpr int kXchBytes = 2 * kTiles * kHalves * kRows * 4;   // [parity][tile][half][row] floats
-constexpr int kSmemBytes = 1024 + kTiles * kQBytes + kStages * 2 * kKVBytes + kNumBars * 8 + 16 + kXchBytes;
+// s_full, p_full, o_done per tile; k/v full, empty per stage
+constexpr int kNumBars = 3 * kTiles + 4 * kStages;
+constexpr int kSmemBytes = 1024 + kTiles * kQBytes + kStages * 2 * kKVBytes + kNumBars * 8 + 16;
 
 // --- tcgen05 wrappers --------------------------------------------------------------
 // Shared-memory matrix descriptor, 128-byte swizzle: start address, leading and stride
@@ -215,10 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
     // S used it, long before P V is done with the V tile beside it
     uint64_t *k_full = bars, *k_empty = bars + kStages, *v_full = bars + 2 * kStages, *v_empty = bars + 3 * kStages;
     uint64_t *s_full = bars + 4 * kStages, *p_full = s_full + kTiles, *o_done = p_full + kTiles;
-    uint64_t *x_bar = o_done + kTiles;                               // [tile][quarter]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float *xch = reinterpret_cast<float *>(tmem_slot + 4);           // 16-byte aligned
 
     const int s = blockIdx.z;
     const int g = blockIdx.y;
@@ -252,9 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
         }
         for (int t = 0; t < kTiles; ++t) {
             mbar_init(&s_full[t], 1);
-            mbar_init(&p_full[t], 4 * kHalves);   // the eight warps of the tile's softmax group
+            mbar_init(&p_full[t], 4);   // the four softmax warps of the tile
             mbar_init(&o_done[t], 1);
-            for (int qq = 0; qq < 4; ++qq) mbar_init(&x_bar[t * 4 + qq], kHalves);
         }
         *abort_flag = 0;
         mbar_fence_init();
@@ -265,16 +260,15 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // softmax warp w: tile (w / 4) % 2, lane quarter w % 4, key / column half w / 8; the
-    // half-0 warps load the query rows (rows past the chunk are zero)
+    // softmax warp w: tile w / 4, lane quarter w % 4; each loads its query row (rows past
+    // the chunk are zero)
     const int quarter = warp & 3;
     const int qtile = (warp >> 2) & 1;
-    const int half = warp >> 3;
     const int row = quarter * 32 + lane;
     const int my_t = t0 + (qtile * kRows + row) / group;
     const int my_h = g * group + row % group;
     const bool row_valid = warp < kSoftmaxWarps && my_t < C;
-    if (warp < kSoftmaxWarps && half == 0) {
+    if (warp < kSoftmaxWarps) {
         const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.q) +
                                                             ((size_t)(q0 + (row_valid ? my_t : 0)) * p.num_q_heads + my_h) * kD);
         unsigned char *dst = sQ + qtile * kQBytes;
@@ -427,23 +421,12 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             __syncwarp();
         }
     } else {
-        // ---------------- softmax of tile qtile, row = TMEM lane, keys / O columns of `half`
+        // ---------------- softmax of tile qtile, one thread per row = TMEM lane
         const bool tile_used = qtile < n_qt;
         const int kmax = row_valid ? P0 + my_t : -1;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const uint32_t s_col = kSCol + qtile * kKeys + half * (kKeys / kHalves);
-        const uint32_t o_col = kOCol + qtile * kD + half * (kD / kHalves);
-        uint64_t *xb = &x_bar[qtile * 4 + quarter];
-        // the partner thread (same row, other half) meets here; a bounded wait
-        auto exchange = [&](int phase, float mine, float &theirs) -> bool {
-            float *x = xch + ((phase & 1) * kTiles + qtile) * kHalves * kRows;
-            x[half * kRows + row] = mine;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(xb);
-            if (!wait_warp(xb, phase & 1, abort_flag)) return false;
-            theirs = x[(1 - half) * kRows + row];
-            return true;
-        };
+        const uint32_t s_col = kSCol + qtile * kKeys;
+        const uint32_t o_col = kOCol + qtile * kD;
         const float sl = p.scale_log2;
         float m = -INFINITY, l = 0.f;
         bool ok = tile_used;
@@ -451,76 +434,49 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             ok = wait_warp(&s_full[qtile], j & 1, abort_flag);
             if (!ok) break;
             fence_after_sync();
-            const int key0 = j * kKeys + half * (kKeys / kHalves);
-            constexpr int kMine = kKeys / kHalves;
+            const int key0 = j * kKeys;
+            // the row's 128 scores: four loads in flight, one wait
+            uint32_t v[kKeys / 32][32];
+#pragma unroll
+            for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(tmem + lane_base + s_col + 32 * c, v[c]);
+            tmem_wait_ld();
             // interior tiles need no mask; the last ones mask by select (keys past this
             // row's position or past the sequence end get weight 0)
-            const bool full_tile = key0 + kMine - 1 <= kmax && key0 + kMine <= L;
-            auto load_chunk = [&](int c, uint32_t (&v)[32]) {
-                tmem_ld32(tmem + lane_base + s_col + 32 * c, v);
-                tmem_wait_ld();
-                if (!full_tile) {
+            if (!(key0 + kKeys - 1 <= kmax && key0 + kKeys <= L)) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int key = key0 + 32 * c + e;
-                        if (!(key <= kmax && key < L)) v[e] = __float_as_uint(-INFINITY);
-                    }
+                for (int e = 0; e < kKeys; ++e) {
+                    const int key = key0 + e;
+                    if (!(key <= kmax && key < L)) v[e >> 5][e & 31] = __float_as_uint(-INFINITY);
                 }
-            };
-            // pass 1: maximum on raw scores (scale > 0 keeps the order), 8 chains
+            }
+            // maximum on raw scores (scale > 0 keeps the order), 8 chains
             float mx8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < kMine / 32; ++c) {
-                uint32_t v[32];
-                load_chunk(c, v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
-            }
-            const float pmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-            float other;
-            ok = exchange(j, pmax, other);
-            if (!ok) break;
-            const float tmax = fmaxf(pmax, other) * sl;     // both halves of the row agree
-            // The rescale decision is taken per warp (tcgen05.ld / st are warp-wide); rows
-            // that do not need it scale by 1.  P_t(j-1) V(j-1) completed before S_t(j)
-            // (issued after it on the same thread), so O_t is settled.
+            for (int e = 0; e < kKeys; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e >> 5][e & 31]));
+            const float tmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl;
+            // The running maximum moves only when a score passes it by 2^8; the O row is
+            // then rescaled by f below, after P is written (the scores are dead by then).
             const bool need = tmax > m + kRescaleThreshold;
-            if (__any_sync(0xffffffffu, need)) {
-                const float f = need ? ex2(m - tmax) : 1.f;
-                if (j > 0) {
-#pragma unroll
-                    for (int c0 = 0; c0 < kD / kHalves; c0 += 32) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_base + o_col + c0, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
-                        tmem_st32(tmem + lane_base + o_col + c0, o);
-                    }
-                    tmem_wait_st();
-                }
-                if (need) {
-                    l *= f;
-                    m = tmax;
-                }
+            const float f = need ? ex2(m - tmax) : 1.f;
+            if (need) {
+                l *= f;
+                m = tmax;
             }
-            // pass 2: p = 2^(s * scale_log2 - m), one FMA and one ex2 per score (-inf -> 0),
-            // written over the chunk's own S columns: per 16 keys, 8 columns of high parts
-            // then 8 of low parts
+            // p = 2^(s * scale_log2 - m), one FMA and one ex2 per score (-inf -> 0), written
+            // over the row's own S columns: per 16 keys, 8 columns of high parts then 8 of
+            // low parts
             const float neg_m = m == -INFINITY ? 0.f : -m;
             float lp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < kMine / 32; ++c) {
-                uint32_t v[32], pw[32];
-                load_chunk(c, v);
+            for (int c = 0; c < kKeys / 32; ++c) {
+                uint32_t pw[32];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float x0 = fmaf(__uint_as_float(v[2 * e]), sl, neg_m);
-                    const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), sl, neg_m);
-                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    const float p0 = ex2(fmaf(__uint_as_float(v[c][2 * e]), sl, neg_m));
+                    const float p1 = ex2(fmaf(__uint_as_float(v[c][2 * e + 1]), sl, neg_m));
                     const int slot = (e >> 3) * 16 + (e & 7);     // key group e/8, pair e%8
                     if (Fmt<T>::two_parts) {
                         // high halves of the two fp32 words = their bf16 truncations; the
@@ -538,21 +494,32 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                 tmem_st32(tmem + lane_base + s_col + 32 * c, pw);
             }
             l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+            // The rescale is warp-wide (tcgen05.ld / st are); rows that do not need it scale
+            // by 1.  P_t(j-1) V(j-1) completed before S_t(j) (issued after it on the same
+            // thread), so O_t is settled, and P_t(j) V(j) waits for this tile's arrival.
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+                for (int c0 = 0; c0 < kD; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_base + o_col + c0, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+                    tmem_st32(tmem + lane_base + o_col + c0, o);
+                }
+            }
             tmem_wait_st();
             fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[qtile]);
         }
         if (ok) ok = wait_warp(&o_done[qtile], (n_tiles - 1) & 1, abort_flag);
-        float l_other = 0.f;
-        if (ok) ok = exchange(n_tiles, l, l_other);       // the row's sum over both halves
         if (ok) {
             fence_after_sync();
-            const float lt = l + l_other;
-            const float inv = lt > 0.f ? 1.f / lt : 0.f;
-            const size_t orow = ((size_t)(q0 + my_t) * p.num_q_heads + my_h) * kD + half * (kD / kHalves);
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const size_t orow = ((size_t)(q0 + my_t) * p.num_q_heads + my_h) * kD;
 #pragma unroll
-            for (int c0 = 0; c0 < kD / kHalves; c0 += 32) {
+            for (int c0 = 0; c0 < kD; c0 += 32) {
                 uint32_t o[32];
                 tmem_ld32(tmem + lane_base + o_col + c0, o);
                 tmem_wait_ld();
