@@ -99,6 +99,13 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
         const int64_t rr = is_v ? r - rows : r;
         const int64_t i = rr / p.num_kv_heads;
         const int h = (int)(rr % p.num_kv_heads);
+        // the row is read before the slot is looked at, so the two loads overlap
+        const unsigned char *src = (is_v ? p.v_new : p.k_new) + (size_t)(rr * D + lane * EPL) * sizeof(T);
+        uint2 u;
+        if constexpr (EPL == 4)
+            u = *reinterpret_cast<const uint2 *>(src);
+        else
+            u.x = *reinterpret_cast<const uint32_t *>(src);
         const int64_t slot = p.slots[i];
         if (slot < 0) continue;
         const int64_t blk = slot / p.block_size;
@@ -107,15 +114,9 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
             if (lane == 0 && !is_v) raise_error(kErrBadSlot);
             continue;
         }
-        const unsigned char *src = (is_v ? p.v_new : p.k_new) + (size_t)(rr * D + lane * EPL) * sizeof(T);
         float x[EPL];
-        if constexpr (EPL == 4) {
-            const uint2 u = *reinterpret_cast<const uint2 *>(src);
-            Elem<T>::widen2(u.x, x);
-            Elem<T>::widen2(u.y, x + 2);
-        } else {
-            Elem<T>::widen2(*reinterpret_cast<const uint32_t *>(src), x);
-        }
+        Elem<T>::widen2(u.x, x);
+        if constexpr (EPL == 4) Elem<T>::widen2(u.y, x + 2);
         uint32_t a = 0;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) a = max(a, __float_as_uint(x[e]) & 0x7fffffffu);

@@ -1155,25 +1155,32 @@ struct AppendParams {
     int64_t num_blocks;
 };
 
-__global__ void __launch_bounds__(128) append_kv_kernel(const AppendParams p) {
-    const int chunks = p.num_kv_heads * p.row_chunks;   // 16-byte chunks per token
-    for (int i = blockIdx.x; i < p.n_tokens; i += gridDim.x) {
+// One thread per 16-byte chunk of a new row (all tokens, heads and chunks flattened,
+// grid-stride): the source read does not wait for the slot, so every thread has its
+// loads in flight at once and the copy runs at memory speed even for a few thousand
+// admitted prompt rows.
+__global__ void __launch_bounds__(256) append_kv_kernel(const AppendParams p) {
+    const int64_t chunks = (int64_t)p.num_kv_heads * p.row_chunks;   // 16-byte chunks per token
+    const int64_t total = (int64_t)p.n_tokens * chunks;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total; g += stride) {
+        const int64_t i = g / chunks;
+        const int t = (int)(g - i * chunks);
+        const uint4 kx = reinterpret_cast<const uint4 *>(p.k_new)[g];   // [n][Hkv][row_chunks]
+        const uint4 vx = reinterpret_cast<const uint4 *>(p.v_new)[g];
         const int64_t slot = p.slots[i];
-        if (slot < 0) continue;
+        if (slot < 0) continue;                                            // padding row
         const int64_t blk = slot / p.block_size;
         const int off = (int)(slot % p.block_size);
         if (blk >= p.num_blocks) {
-            if (threadIdx.x == 0) raise_error(kErrBadSlot);
+            if (t == 0) raise_error(kErrBadSlot);
             continue;
         }
-        for (int t = threadIdx.x; t < chunks; t += blockDim.x) {
-            const int h = t / p.row_chunks;
-            const int c = t % p.row_chunks;
-            const size_t dst = (((size_t)blk * p.num_kv_heads + h) * p.block_size + off) * p.row_chunks + c;
-            const size_t src = ((size_t)i * p.num_kv_heads + h) * p.row_chunks + c;
-            reinterpret_cast<uint4 *>(p.k_layer)[dst] = reinterpret_cast<const uint4 *>(p.k_new)[src];
-            reinterpret_cast<uint4 *>(p.v_layer)[dst] = reinterpret_cast<const uint4 *>(p.v_new)[src];
-        }
+        const int h = t / p.row_chunks;
+        const int c = t - h * p.row_chunks;
+        const size_t dst = (((size_t)blk * p.num_kv_heads + h) * p.block_size + off) * p.row_chunks + c;
+        reinterpret_cast<uint4 *>(p.k_layer)[dst] = kx;
+        reinterpret_cast<uint4 *>(p.v_layer)[dst] = vx;
     }
 }
 
@@ -1780,8 +1787,9 @@ pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const vo
     p.num_kv_heads = pool->cfg.num_kv_heads;
     p.row_chunks = (int32_t)(row_bytes / 16);
     p.num_blocks = pool->cfg.num_blocks;
-    const int grid = n_tokens < 148 * 32 ? n_tokens : 148 * 32;
-    append_kv_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    const int64_t threads = (int64_t)n_tokens * p.num_kv_heads * p.row_chunks;
+    const int grid = (int)std::min<int64_t>((threads + 255) / 256, 148 * 16);
+    append_kv_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
     pa_internal::launch_count.fetch_add(1);
     return check_launch("append_kv_kernel");
 }
