@@ -60,7 +60,7 @@ def parse(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--repeats", type=int, default=None,
                     help="timed passes of --steps steps each, over a longer schedule; the median pass is "
-                         "reported (default 7; 3 for large_pool)")
+                         "reported (default 7 on the continuous batches, 3 on the fixed batches)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="continuous_batch", choices=WORKLOADS)
     ap.add_argument("--split", type=int, default=None, help="tokens per split-K range (0: never split)")
@@ -81,7 +81,8 @@ def parse(argv=None):
     if a.split is None:
         a.split = default_split(a.workload)
     if a.repeats is None:
-        a.repeats = 3 if a.workload.startswith("large_pool") else 7
+        # 3 passes where one step is long (large pool) or sequences only grow (fixed batches)
+        a.repeats = 7 if a.workload in ("continuous_batch", "shared_prompt") else 3
     a.repeats = max(1, a.repeats)
     if a.kv_dtype == "fp8" and a.workload not in ("continuous_batch", "large_pool_b16", "large_pool_b32",
                                                     "worked_example"):
@@ -136,13 +137,15 @@ def make_recipe(workload, seed_offset, steps):
     from synthetic import workloads as wl
     if workload == "continuous_batch":
         return wl.continuous_batch(seed=3 + seed_offset, steps=steps)
+    # the fixed-batch workloads grow by one token per sequence and step: their pools get
+    # room for every step the run takes
     if workload.startswith("large_pool"):
-        return wl.large_pool(seed=5 + seed_offset, block_size=int(workload[-2:]))
+        return wl.large_pool(seed=5 + seed_offset, block_size=int(workload[-2:]), steps=steps)
     if workload == "worked_example":
-        return wl.worked_example(seed=2 + seed_offset)
+        return wl.worked_example(seed=2 + seed_offset, steps=steps)
     if workload == "shared_prompt":
         return wl.shared_prompt_batch(seed=6 + seed_offset, steps=steps)
-    return wl.prefix_sharing(seed=4 + seed_offset)
+    return wl.prefix_sharing(seed=4 + seed_offset, steps=steps)
 
 
 # Workloads whose KV (or unique KV) per step fits in the 126 MB L2: each step starts by

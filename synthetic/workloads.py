@@ -37,10 +37,11 @@ def tiny(seed: int = 1) -> dict:
                 order=rng.permutation(shape.num_blocks).astype(np.int32))
 
 
-def worked_example(seed: int = 2) -> dict:
-    """The pages' four requests (3900/420/2100/70 tokens), 32 q / 8 KV heads, d128, fp16."""
+def worked_example(seed: int = 2, steps: int = 0) -> dict:
+    """The pages' four requests (3900/420/2100/70 tokens), 32 q / 8 KV heads, d128, fp16.
+    ``steps``: decode steps the pool must also hold (each appends one token per request)."""
     rng = np.random.default_rng(seed)
-    shape = Shape(1, 16, 32, 8, 128, "f16", 4096, kv_scale=1.0 / math.sqrt(128.0))
+    shape = Shape(1, 16, 32, 8, 128, "f16", 4096 + 4 * -(-steps // 16), kv_scale=1.0 / math.sqrt(128.0))
     return dict(name="worked_example", seed=seed, shape=shape,
                 lens=np.array([3900, 420, 2100, 70]),
                 order=rng.permutation(shape.num_blocks).astype(np.int32))
@@ -87,11 +88,12 @@ def continuous_batch(seed: int = 3, n: int = 256, steps: int = 64, p_stop: float
                 schedule=continuous_schedule(n, steps, seed, lo, hi, p_stop))
 
 
-def prefix_sharing(seed: int = 4, n: int = 64, prefix: int = 2048) -> dict:
-    """64 sequences sharing a 2048-token prefix, private suffixes U[16, 512], fp16."""
+def prefix_sharing(seed: int = 4, n: int = 64, prefix: int = 2048, steps: int = 0) -> dict:
+    """64 sequences sharing a 2048-token prefix, private suffixes U[16, 512], fp16.
+    ``steps``: decode steps beyond the first few the pool must also hold."""
     rng = np.random.default_rng(seed)
     shape = Shape(1, 16, 32, 8, 128, "f16",
-                  num_blocks=prefix // 16 + n * ((512 + 16 + 15) // 16 + 1) + 64,
+                  num_blocks=prefix // 16 + n * ((512 + 16 + 15) // 16 + 1 + -(-steps // 16)) + 64,
                   kv_scale=1.0 / math.sqrt(128.0))
     suffix = rng.integers(16, 512 + 1, size=n)
     order = rng.permutation(shape.num_blocks).astype(np.int32)
@@ -107,11 +109,13 @@ def lognormal_lengths(n: int, seed: int, median: float = 1500.0, sigma: float = 
     return np.clip(lens, 1, cap).astype(np.int64)
 
 
-def large_pool(seed: int = 5, block_size: int = 16, n: int = 384, num_layers: int = 32) -> dict:
-    """384 sequences, lognormal lengths (median 1500, sigma 0.75, cap 16384), 32 layers, fp16."""
+def large_pool(seed: int = 5, block_size: int = 16, n: int = 384, num_layers: int = 32, steps: int = 0) -> dict:
+    """384 sequences, lognormal lengths (median 1500, sigma 0.75, cap 16384), 32 layers, fp16.
+    ``steps``: decode steps the pool must also hold (one token per sequence each)."""
     lens = lognormal_lengths(n, seed)
     # pool: every sequence's blocks after one appended token, plus two blocks of headroom each
-    nb = int(sum(-(-(int(l) + 1) // block_size) for l in lens)) + 2 * n
+    # (and room for ``steps`` more tokens per sequence)
+    nb = int(sum(-(-(int(l) + 1 + steps) // block_size) for l in lens)) + 2 * n
     shape = Shape(num_layers, block_size, 32, 8, 128, "f16", nb, kv_scale=1.0 / math.sqrt(128.0))
     order = np.random.default_rng(seed + 1000 * block_size).permutation(nb).astype(np.int32)
     return dict(name=f"large_pool_b{block_size}", seed=seed, shape=shape, lens=lens, order=order)
