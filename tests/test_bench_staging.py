@@ -1,6 +1,7 @@
 """Host-side staging of bench.py on CPU: the packed layouts that let one copy upload a
 step's metadata (and, end to end, a layer's q/K/V and prompt rows)."""
 import numpy as np
+import pytest
 import torch
 
 import bench
@@ -60,3 +61,21 @@ def test_empty_prompt_part():
     assert v["pk"].shape == (0, 2, 8) and v["pv"].numel() == 0
     assert p.end["q"] == 4 * 2 * 8 * 2 and p.off["pk"] == bench.Packed.ALIGN
     assert p.end["pv"] == p.off["pv"] == p.off["pk"]
+
+
+@pytest.mark.parametrize("workload", ["large_pool_b16", "large_pool_b32", "prefix_sharing", "worked_example"])
+def test_fixed_batch_pools_hold_every_step_of_a_run(workload):
+    """A fixed batch grows by one token per sequence and step; the benchmark's default run
+    (warm-up, every timed pass, the end-to-end passes) must fit its pool."""
+    import bench
+    a = bench.parse(["--workload", workload])
+    total = a.warmup + a.repeats * a.steps + min(a.repeats, 3) * a.steps
+    r = bench.make_recipe(workload, 0, total)
+    sh = r["shape"]
+    B = sh.block_size
+    if workload == "prefix_sharing":
+        shared = r["prefix"] // B
+        need = shared + sum(-(-(r["prefix"] + int(x) + total) // B) - shared for x in r["suffix"])
+    else:
+        need = sum(-(-(int(L) + total) // B) for L in r["lens"])
+    assert need <= sh.num_blocks, (need, sh.num_blocks)
