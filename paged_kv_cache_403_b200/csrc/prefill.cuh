@@ -180,6 +180,27 @@ struct Fmt<__nv_bfloat16> {
     static constexpr bool two_parts = true;
 };
 
+// Pairs of fp32 values in one 64-bit register (element 0 in the low half) and the packed
+// fp32x2 arithmetic of sm_100, which does two fp32 operations per instruction.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t byte_perm(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
@@ -469,31 +490,44 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             // over the row's own S columns: per 16 keys, 8 columns of high parts then 8 of
             // low parts
             const float neg_m = m == -INFINITY ? 0.f : -m;
-            float lp[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint64_t sl2 = f32x2(sl, sl), nm2 = f32x2(neg_m, neg_m);
+            uint64_t lp2[2] = {0ull, 0ull};                   // two pairs of running sums
 #pragma unroll
             for (int c = 0; c < kKeys / 32; ++c) {
                 uint32_t pw[32];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(__uint_as_float(v[c][2 * e]), sl, neg_m));
-                    const float p1 = ex2(fmaf(__uint_as_float(v[c][2 * e + 1]), sl, neg_m));
+                    float x0, x1;
+                    unpack_f32x2(fma_f32x2(f32x2(__uint_as_float(v[c][2 * e]), __uint_as_float(v[c][2 * e + 1])), sl2,
+                                           nm2),
+                                 x0, x1);
+                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    const uint64_t p2 = f32x2(p0, p1);
                     const int slot = (e >> 3) * 16 + (e & 7);     // key group e/8, pair e%8
                     if (Fmt<T>::two_parts) {
                         // high halves of the two fp32 words = their bf16 truncations; the
                         // remainders (exact in fp32, >= 0) truncated the same way
                         const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
                         pw[slot] = byte_perm(b0, b1, 0x7632u);
-                        pw[slot + 8] = byte_perm(__float_as_uint(p0 - __uint_as_float(b0 & 0xffff0000u)),
-                                                 __float_as_uint(p1 - __uint_as_float(b1 & 0xffff0000u)), 0x7632u);
+                        float r0, r1;
+                        unpack_f32x2(add_f32x2(p2, f32x2(__uint_as_float((b0 & 0xffff0000u) ^ 0x80000000u),
+                                                         __uint_as_float((b1 & 0xffff0000u) ^ 0x80000000u))),
+                                     r0, r1);
+                        pw[slot + 8] = byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632u);
                     } else {
                         pw[slot] = Mma<T>::pack(p0, p1);
                         pw[slot + 8] = 0u;
                     }
-                    lp[e & 3] += p0 + p1;
+                    lp2[e & 1] = add_f32x2(lp2[e & 1], p2);
                 }
                 tmem_st32(tmem + lane_base + s_col + 32 * c, pw);
             }
-            l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+            {
+                float a0, a1, b0, b1;
+                unpack_f32x2(lp2[0], a0, a1);
+                unpack_f32x2(lp2[1], b0, b1);
+                l += (a0 + a1) + (b0 + b1);
+            }
             // The rescale is warp-wide (tcgen05.ld / st are); rows that do not need it scale
             // by 1.  P_t(j-1) V(j-1) completed before S_t(j) (issued after it on the same
             // thread), so O_t is settled, and P_t(j) V(j) waits for this tile's arrival.
