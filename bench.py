@@ -665,7 +665,7 @@ def run_ours(args):
                                    + " (+ plan_kernel; split partials merged in the kernel)",
                          "attn_ms_mean": round(attn_mean_ms, 4), "alg_bytes_per_launch": int(alg_per_launch),
                          "launches_timed": len(attn_ms), "peak_source": peak_src},
-            "gpu_launches": int(launches),
+            "gpu_launches": int(round(launches)),   # per timed pass (mean over the passes)
             "host_ms_per_step": round(host_ms, 4),
             "device_error": pa.pa_device_error(),
             "clocks": clk,
