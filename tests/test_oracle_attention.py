@@ -318,3 +318,18 @@ def test_pins_reject_planted_mistake(name):
             % (here, os.path.dirname(here), so))
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, timeout=300)
     assert r.returncode != 0, f"mutant {name} passed every pin"
+
+
+def test_whole_batch_helper_matches_per_sequence_helper():
+    """The full-size GPU checks attend over a whole batch's regenerated histories in one
+    oracle call; each row must equal the per-sequence oracle call bit for bit."""
+    from oracle_replay import histories_attention, sequence_attention
+    from synthetic import workloads as wl
+    r = wl.worked_example()
+    sh = r["shape"]
+    uids, lens = [3, 9, 1, 4], [70, 17, 33, 1]
+    pos = [L - 1 for L in lens]
+    batch = histories_attention(sh, r["seed"], 0, uids, lens, pos)
+    for i in range(4):
+        one = sequence_attention(sh, r["seed"], 0, uids[i], lens[i], uids[i], pos[i])
+        assert np.array_equal(batch[i], one)
