@@ -1156,9 +1156,8 @@ struct AppendParams {
 };
 
 // One thread per 16-byte chunk of a new row (all tokens, heads and chunks flattened,
-// grid-stride): the source read does not wait for the slot, so every thread has its
-// loads in flight at once and the copy runs at memory speed even for a few thousand
-// admitted prompt rows.
+// grid-stride); the source read is issued before the slot lookup, so a thread's loads
+// are in flight together.
 __global__ void __launch_bounds__(256) append_kv_kernel(const AppendParams p) {
     const int64_t chunks = (int64_t)p.num_kv_heads * p.row_chunks;   // 16-byte chunks per token
     const int64_t total = (int64_t)p.n_tokens * chunks;
