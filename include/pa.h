@@ -363,12 +363,14 @@ uint64_t pa_launch_count(void);
  * than stall -- only motivate it).  Every device-side wait of the library's kernels
  * is bounded; this sets the bound on the current device to wait_limit_ns
  * (<= 0 restores the default of 2 s) and, when withhold_cta >= 0, makes the
- * producer warp of the decode CTA with that linear block index issue no copies
- * (every later pa_decode_attention launch on any device, until called again with
- * -1).  That CTA's consumers then wait for data that never comes: each wait runs
- * out after the bound, records device error bit 4 and returns, no copy is left in
- * flight, and the rest of the launch is unaffected; the withheld CTA's outputs are
- * not meaningful.  Off by default; synchronises the device. */
+ * producer warp of the CTA with that linear block index issue no copies (every
+ * later pa_decode_attention and pa_prefill_attention launch on any device, until
+ * called again with -1).  That CTA's other warps then wait for data that never
+ * comes: each wait runs out after the bound, records device error bit 4 and
+ * returns (the prefill kernel's roles also share an abort flag, and its tensor
+ * memory is still freed), no copy is left in flight, and the rest of the launch is
+ * unaffected; the withheld CTA's outputs are not meaningful.  Off by default;
+ * synchronises the device. */
 pa_status pa_debug_wait_test(int64_t wait_limit_ns, int32_t withhold_cta);
 
 #ifdef __cplusplus

@@ -99,8 +99,9 @@ __device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
 
 __device__ __forceinline__ uint64_t wait_limit_ns() { return *static_cast<volatile uint64_t *>(&g_wait_limit_ns); }
 
-// A wait-expiry test (pa_debug_wait_test) names one decode CTA, by its linear block
-// index, whose producer issues no copies, so that its consumers' waits run out.
+// A wait-expiry test (pa_debug_wait_test) names one decode or prefill CTA, by its
+// linear block index, whose producer issues no copies, so that the waits of its other
+// warps run out.
 __device__ __forceinline__ bool copies_withheld(int32_t withhold) {
     return withhold >= 0 &&
            (int64_t)blockIdx.x + (int64_t)gridDim.x * (blockIdx.y + (int64_t)gridDim.y * blockIdx.z) == withhold;
@@ -1410,7 +1411,8 @@ pa_status launch_prefill(const prefill::Params &p, dim3 grid, cudaStream_t strea
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// Decode CTA whose copies a wait-expiry test withholds (pa_debug_wait_test), else -1.
+// Decode or prefill CTA whose copies a wait-expiry test withholds (pa_debug_wait_test),
+// else -1.
 std::atomic<int32_t> g_debug_withhold{-1};
 
 // Decode workspace: split partials (acc [parts][D] then (m, l) [parts][2], fp32) when a
@@ -1721,6 +1723,7 @@ pa_status pa_prefill_attention(pa_pool *pool, int32_t layer, const void *q, void
     p.block_size = c.block_size;
     p.out_f32 = out_dtype == PA_F32;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.debug_withhold = g_debug_withhold.load(std::memory_order_relaxed);
     const dim3 grid((unsigned)tiles, c.num_kv_heads, n_seqs);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (c.dtype == PA_BF16)

@@ -217,6 +217,7 @@ struct Params {
     const int32_t *lens;        // [n] total tokens (context + chunk)
     const int32_t *q_start;     // [n + 1]
     int32_t max_blocks, num_blocks, num_kv_heads, num_q_heads, layer, block_size, out_f32;
+    int32_t debug_withhold;     // see copies_withheld(); -1 outside wait-expiry tests
     float scale_log2;
 };
 
@@ -310,7 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
         // ---------------- producer: walk the table, keep the ring full
         const int32_t *trow = p.tables + (size_t)s * p.max_blocks;
         int issued_k = 0, issued_v = 0;   // tiles whose K / V copies were issued
-        for (int j = 0; j < n_tiles; ++j) {
+        // a wait-expiry test withholds every copy of one CTA: its other roles' waits run out
+        const int to_issue = copies_withheld(p.debug_withhold) ? 0 : n_tiles;
+        for (int j = 0; j < to_issue; ++j) {
             const int st = j % kStages;
             int blk = 0;
             if (lane < BLOCKS_PER_TILE) {

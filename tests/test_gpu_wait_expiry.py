@@ -89,3 +89,31 @@ def test_hook_rejects_bad_arguments():
     with pytest.raises(pa.PaError) as e:
         pa.pa_debug_wait_test(0, -2)
     assert e.value.status == pa.PA_ERR_INVALID_ARG
+
+
+def test_prefill_withheld_copies_time_out_and_report():
+    """The same on the tcgen05 chunked-prefill kernel, whose TMA, tensor-core and softmax
+    roles hand tiles to each other through mbarriers: with CTA 0's copies withheld its
+    tensor-core warp's wait for the first key tile runs out, the shared abort flag
+    releases the softmax warps, the CTA frees its tensor memory and ends; its output rows
+    are left untouched and every other CTA's rows are exactly the normal ones."""
+    from test_gpu_prefill import prefill_case, run
+    c = prefill_case([600, 300], [200, 129], seed=21)   # group 4: 64 tokens x 4 heads per CTA
+    normal = run(c)
+    assert pa.pa_device_error(clear=True) == 0
+    pa.pa_debug_wait_test(1_000_000, 0)
+    try:
+        failed = run(c)                                  # outputs start as NaN
+        code = pa.pa_device_error(clear=True)
+    finally:
+        pa.pa_debug_wait_test(0, -1)
+    assert code & ERR_TIMEOUT, f"device error word {code:#x}: the withheld CTA's waits did not report"
+    # CTA 0 = sequence 0, KV head 0 (query heads 0-3), the chunk's first 64 tokens (rows 0-63)
+    mine = np.zeros(failed.shape[:2], bool)
+    mine[0:64, 0:4] = True
+    assert np.isnan(failed[mine]).all()
+    assert np.array_equal(failed[~mine], normal[~mine])
+    again = run(c)
+    assert pa.pa_device_error(clear=True) == 0
+    assert np.array_equal(again, normal)
+    check_close(again, c["ref"], "f32", "bf16", "prefill after the hook is off")
