@@ -21,20 +21,23 @@
 //                    running maximum by 2^8), and P written back to TMEM (tcgen05.st) as
 //                    the A operand of P V: for bf16 a truncated high part plus the
 //                    truncated remainder, for fp16 once;
-//   warp 8           tensor-core issue (one lane): S_t = Q_t K^T (M=128, N=128 keys,
+//   warp 8           tensor-core issue, one thread: S_t = Q_t K^T (M=128, N=128 keys,
 //                    both operands in shared memory) and O_t += P_t V (M=128,
 //                    N=head_dim, per part of P; A = P from TMEM, B = V from shared
-//                    memory);
+//                    memory).  The tensor core keeps almost no queue of its own, so this
+//                    thread does nothing but wait and issue: a cycle it spends elsewhere
+//                    is a cycle the tensor core idles;
 //   warp 9           TMA producer: 128-key tiles of K and V (2-D tensor loads, 128-byte
-//                    swizzle) into a 2-stage ring, walking the block table.
-// Tiles of 128 keys make S = Q K^T an M=128, N=128 product: at N=64 the tensor core ran
-// it at about a third of its rate.  TMEM then holds O and S of both query tiles (512
+//                    swizzle) into a 2-stage ring, walking the block table; it also zeroes
+//                    the last value tile's rows past the sequence end.
+// Tiles of 128 keys make S = Q K^T an M=128, N=128 product (64 cycles at the dense
+// rate; an N=64 product takes 48, two thirds of that rate).  TMEM then holds O and S of both query tiles (512
 // columns), so P is written over S in place: the 16 columns of each 16-key group of S
 // take that group's P (8 columns of high parts, 8 of low parts), and the next S of the
 // tile is issued after the P V that reads them (one thread's tcgen05.mma run in order).
 // The two tiles ping-pong: while one tile's softmax computes exponentials the tensor
 // core works on the other tile.  Every hand-off is an mbarrier; every wait is bounded and
-// sets a shared abort flag that all roles check; TMEM is always freed.  Key rows past
+// sets a shared abort flag that all roles check; TMEM is always freed.  Value rows past
 // the sequence end are zeroed in shared memory before P V (weight 0, but 0 * NaN would
 // not be 0).
 namespace prefill {
@@ -54,8 +57,9 @@ constexpr uint32_t kOCol = 0, kSCol = 256;
 constexpr int kQBytes = kRows * kD * 2;         // 32 KB per tile: [2 halves][128 rows][128 B]
 constexpr int kKVBytes = kKeys * kD * 2;        // 32 KB: [2 halves][128 rows][128 B]
 constexpr int kStages = 2;
-// s_full, p_full, o_done per tile; k/v full, empty per stage
-constexpr int kNumBars = 3 * kTiles + 4 * kStages;
+// s_full, p_full, o_done per tile; k/v full, empty per stage; v_fixed (the last value
+// tile after its rows past the sequence end were zeroed)
+constexpr int kNumBars = 3 * kTiles + 4 * kStages + 1;
 constexpr int kSmemBytes = 1024 + kTiles * kQBytes + kStages * 2 * kKVBytes + kNumBars * 8 + 16;
 
 // --- tcgen05 wrappers --------------------------------------------------------------
@@ -162,6 +166,23 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// The same for one thread (the tensor-core issuer): the tensor core's queue is short, so
+// every cycle this thread spends outside tcgen05.mma is a cycle the tensor core may idle.
+__device__ __forceinline__ bool wait_one(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns(), limit = wait_limit_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag || global_timer_ns() - t0 > limit) {
+            if (!*abort_flag) {
+                raise_error(kErrTimeout);
+                *abort_flag = 1;
+            }
+            return false;
+        }
+    }
+    return true;
+}
+
 // Operand format code of the instruction descriptor, and how P enters P V: bf16 P
 // keeps 8 significant bits, too few for the 2e-3 bound on peaky rows, so a bf16 P is a
 // high part (the truncation of p to bf16) plus the truncation of the exact remainder
@@ -235,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
     // S used it, long before P V is done with the V tile beside it
     uint64_t *k_full = bars, *k_empty = bars + kStages, *v_full = bars + 2 * kStages, *v_empty = bars + 3 * kStages;
     uint64_t *s_full = bars + 4 * kStages, *p_full = s_full + kTiles, *o_done = p_full + kTiles;
+    uint64_t *v_fixed = o_done + kTiles;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -273,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             mbar_init(&p_full[t], 4);   // the four softmax warps of the tile
             mbar_init(&o_done[t], 1);
         }
+        mbar_init(v_fixed, 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -348,6 +371,26 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
             if (*abort_flag) break;
             __syncwarp();
         }
+        // Value rows past the sequence end (only the last tile has any) are zeroed here, once
+        // that tile's copy has landed, and handed to the tensor-core thread through v_fixed:
+        // their weights are 0, but 0 * NaN would not be 0.
+        const int last = n_tiles - 1;
+        const int first_bad = L - last * kKeys;
+        if (issued_v == n_tiles && first_bad < kKeys &&
+            wait_warp(&v_full[last % kStages], (last / kStages) & 1, abort_flag)) {
+            unsigned char *v_st = sKV + (last % kStages) * 2 * kKVBytes + kKVBytes;
+            for (int rr = lane; rr < 2 * kKeys; rr += 32) {
+                const int r = rr >> 1, half = rr & 1;
+                if (r >= first_bad) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(v_st + half * (kKVBytes / 2) + r * 128);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(v_fixed);
+        }
         // every issued copy lands before the CTA frees its shared memory, also after an abort
         if (lane == 0) {
             drain_copies(k_full, issued_k, kStages);
@@ -355,43 +398,28 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
-        // ---------------- tensor-core issue
-        // wait for tile j's keys
-        auto ready_k = [&](int j) -> bool {
-            if (!wait_warp(&k_full[j % kStages], (j / kStages) & 1, abort_flag)) return false;
-            fence_after_sync();
-            return true;
-        };
-        // wait for tile j's values; zero value rows past the sequence end
-        auto ready_v = [&](int j) -> bool {
-            const int st = j % kStages;
-            if (!wait_warp(&v_full[st], (j / kStages) & 1, abort_flag)) return false;
-            const int first_bad = L - j * kKeys;
-            if (first_bad < kKeys) {
-                unsigned char *v_st = sKV + st * 2 * kKVBytes + kKVBytes;
-                for (int rr = lane; rr < 2 * kKeys; rr += 32) {
-                    const int r = rr >> 1, half = rr & 1;
-                    if (r >= first_bad) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(v_st + half * (kKVBytes / 2) + r * 128);
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-                    }
-                }
-                fence_proxy_async();
-                __syncwarp();
-            }
-            fence_after_sync();
-            return true;
-        };
-        // Descriptors are built once: the start address sits in the low 14 bits as
-        // addr >> 4 (shared memory < 256 KB), so moving to another tile, stage or K step
-        // is one add of offset >> 4 -- a freshly built descriptor per instruction left the
-        // issuing lane, not the tensor core, as the bottleneck.
-        const uint64_t q_desc = smem_desc(smem_addr(sQ), 16, 1024);
-        const uint64_t k_desc = smem_desc(smem_addr(sKV), 16, 1024);
-        const uint64_t v_desc = smem_desc(smem_addr(sKV + kKVBytes), kKVBytes / 2, 1024);
-        auto issue_s = [&](int t, int j) {
-            if (lane == 0) {
+        // ---------------- tensor-core issue, one thread (the others wait at the end)
+        if (lane == 0) {
+            const int last = n_tiles - 1;
+            const bool fixed_last = L - last * kKeys < kKeys;   // the producer zeroes its tail rows
+            auto ready_k = [&](int j) -> bool {
+                if (!wait_one(&k_full[j % kStages], (j / kStages) & 1, abort_flag)) return false;
+                fence_after_sync();
+                return true;
+            };
+            auto ready_v = [&](int j) -> bool {
+                if (!wait_one(&v_full[j % kStages], (j / kStages) & 1, abort_flag)) return false;
+                if (j == last && fixed_last && !wait_one(v_fixed, 0, abort_flag)) return false;
+                fence_after_sync();
+                return true;
+            };
+            // Descriptors are built once: the start address sits in the low 14 bits as
+            // addr >> 4 (shared memory < 256 KB), so moving to another tile, stage or K step
+            // is one add of offset >> 4.
+            const uint64_t q_desc = smem_desc(smem_addr(sQ), 16, 1024);
+            const uint64_t k_desc = smem_desc(smem_addr(sKV), 16, 1024);
+            const uint64_t v_desc = smem_desc(smem_addr(sKV + kKVBytes), kKVBytes / 2, 1024);
+            auto issue_s = [&](int t, int j) {
                 const uint64_t qa = q_desc + (uint64_t)((t * kQBytes) >> 4);
                 const uint64_t kb = k_desc + (uint64_t)(((j % kStages) * 2 * kKVBytes) >> 4);
 #pragma unroll
@@ -401,11 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                     umma(tmem + kSCol + t * kKeys, qa + qo, kb + ko, IDESC_S, kk > 0);
                 }
                 umma_commit(&s_full[t]);
-            }
-            __syncwarp();
-        };
-        auto issue_pv = [&](int t, int j) {
-            if (lane == 0) {
+            };
+            auto issue_pv = [&](int t, int j) {
                 const uint32_t pcol = tmem + kSCol + t * kKeys;
                 const uint64_t vb = v_desc + (uint64_t)(((j % kStages) * 2 * kKVBytes) >> 4);
 #pragma unroll
@@ -415,35 +440,30 @@ __global__ void __launch_bounds__(kThreads, 1) paged_prefill_kernel(const __grid
                     if (Fmt<T>::two_parts) umma_ts(tmem + kOCol + t * kD, pcol + kk * 16 + 8, b, IDESC_O, 1u);
                 }
                 umma_commit(&o_done[t]);
+            };
+            bool ok = ready_k(0);
+            if (ok) {
+                for (int t = 0; t < n_qt; ++t) issue_s(t, 0);
+                umma_commit(&k_empty[0]);   // K(0) free once both S(0) are done
             }
-            __syncwarp();
-        };
-        bool ok = ready_k(0);
-        if (ok) {
-            for (int t = 0; t < n_qt; ++t) issue_s(t, 0);
-            if (lane == 0) umma_commit(&k_empty[0]);   // K(0) free once both S(0) are done
-            __syncwarp();
-        }
-        for (int j = 0; j < n_tiles && ok; ++j) {
-            for (int t = 0; t < n_qt && ok; ++t) {
-                ok = wait_warp(&p_full[t], j & 1, abort_flag);   // softmax t read S_t(j), wrote P_t(j)
-                if (!ok) break;
-                fence_after_sync();
-                // P_t(j) V(j) first: S_t(j+1) overwrites the columns P_t(j) is read from
-                if (t == 0) ok = ready_v(j);
-                if (!ok) break;
-                issue_pv(t, j);
-                if (j + 1 < n_tiles) {
-                    if (t == 0) ok = ready_k(j + 1);
-                    if (ok) issue_s(t, j + 1);
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                for (int t = 0; t < n_qt; ++t) {
+                    // softmax t read S_t(j) and wrote P_t(j)
+                    if (!(ok = wait_one(&p_full[t], j & 1, abort_flag))) break;
+                    fence_after_sync();
+                    if (t == 0 && !(ok = ready_v(j))) break;
+                    // P_t(j) V(j) first: S_t(j+1) overwrites the columns P_t(j) is read from
+                    issue_pv(t, j);
+                    if (t == n_qt - 1) umma_commit(&v_empty[j % kStages]);   // V(j) read for the last time
+                    if (j + 1 < n_tiles) {
+                        if (t == 0 && !(ok = ready_k(j + 1))) break;
+                        issue_s(t, j + 1);
+                    }
                 }
+                if (ok && j + 1 < n_tiles) umma_commit(&k_empty[(j + 1) % kStages]);
             }
-            if (ok && lane == 0) {
-                umma_commit(&v_empty[j % kStages]);
-                if (j + 1 < n_tiles) umma_commit(&k_empty[(j + 1) % kStages]);
-            }
-            __syncwarp();
         }
+        __syncwarp();
     } else {
         // ---------------- softmax of tile qtile, one thread per row = TMEM lane
         const bool tile_used = qtile < n_qt;
