@@ -351,14 +351,15 @@ class Replica:
         # reservation and table calls then pass pointers without converting lists
         self.sid_arr = np.asarray(self.sids, np.int32)
         self.ones = np.ones(n, np.int32)
-        # every step's inputs (all layers), generated on the device before any timing
+        # every step's inputs (all layers), generated on the device before any timing: q, and
+        # the K / V rows to append -- the step's token rows with the admitted prompts' rows
+        # right after them, so that one append launch writes both
         self.inputs = []
         for st in self.plan:
             per_layer = []
             for layer in range(self.NL):
                 k, v = gen.kv(layer, st["uids"], st["pos"])
                 q = gen.q(layer, st["uids"], st["pos"])
-                pk = pv = None
                 if st["admitted"]:
                     if workload == "shared_prompt":
                         u, tk = map(np.concatenate, zip(*[self.prompt_rows(uid, p) for _, uid, p in st["admitted"]]))
@@ -366,49 +367,51 @@ class Replica:
                         u = np.concatenate([np.full(p, uid) for _, uid, p in st["admitted"]])
                         tk = np.concatenate([np.arange(p) for _, _, p in st["admitted"]])
                     pk, pv = gen.kv(layer, u, tk)
-                per_layer.append((q, k, v, pk, pv))
+                    k, v = torch.cat([k, pk]), torch.cat([v, pv])
+                per_layer.append((q, k, v))
             self.inputs.append(per_layer)
         torch.cuda.synchronize()
-        # end-to-end leg: each (step, layer)'s q, K, V rows and prompt rows packed in one
-        # pinned host buffer; one copy per layer uploads them into a device buffer of the
-        # same layout (prompt rows right after the step's own rows, so only the rows of
-        # this step's admissions cross the bus)
+        # end-to-end leg: each (step, layer)'s q and K / V rows (token rows, then the admitted
+        # prompts' rows) packed in one pinned host buffer; one copy per layer uploads them
+        # into a device buffer of the same layout (sized per step, so only the rows of this
+        # step's admissions cross the bus)
         self.host, self.e2e_views, self.e2e_bytes = {}, {}, {}
         dt = self.inputs[0][0][0].dtype
         row_shape = lambda rows: (rows, sh.num_kv_heads, sh.head_dim)  # noqa: E731
         self.e2e_layout = {}
         if e2e_from is not None:
             for t in range(e2e_from, total_steps):
-                ptot_t = 0 if self.inputs[t][0][3] is None else self.inputs[t][0][3].shape[0]
-                lay = Packed([("q", dt, (n, sh.num_q_heads, sh.head_dim)), ("k", dt, row_shape(n)),
-                              ("v", dt, row_shape(n)), ("pk", dt, row_shape(ptot_t)), ("pv", dt, row_shape(ptot_t))])
+                rows_t = self.inputs[t][0][1].shape[0]
+                lay = Packed([("q", dt, (n, sh.num_q_heads, sh.head_dim)), ("k", dt, row_shape(rows_t)),
+                              ("v", dt, row_shape(rows_t))])
                 self.e2e_layout[t] = lay
                 self.host[t] = []
                 for src in self.inputs[t]:
                     buf = torch.empty(lay.nbytes, dtype=torch.uint8).pin_memory()
                     views = lay.views(buf)
-                    for name, x in zip(("q", "k", "v", "pk", "pv"), src):
-                        if x is not None:
-                            views[name].copy_(x)
+                    for name, x in zip(("q", "k", "v"), src):
+                        views[name].copy_(x)
                     self.host[t].append(buf)
-                self.e2e_bytes[t] = lay.end["pv"]
+                self.e2e_bytes[t] = lay.end["v"]
         mb = self.max_blocks
         pin = lambda shape, dt: torch.empty(shape, dtype=dt).pin_memory()  # noqa: E731
         max_prompt = max([sum(p - self.prompt_start(p) for _, _, p in st["admitted"]) for st in self.plan] + [1])
         H, D2 = NSETS + 1, NSETS
-        # one step's metadata, packed so that one copy uploads it (prompt slots last: only
-        # the used ones are copied)
+        # one step's metadata, packed so that one copy uploads it; the slots come last --
+        # the step's n token slots, then the admitted prompts' slots, matching the order of
+        # the rows to append -- and only the used ones are copied
         self.meta = Packed([("tables", torch.int32, (n, mb)), ("lens", torch.int32, (n,)),
-                            ("slots", torch.int64, (n,)), ("cow", torch.int32, (n, 2)),
-                            ("pslots", torch.int64, (max_prompt,))])
+                            ("cow", torch.int32, (n, 2)), ("slots", torch.int64, (n + max_prompt,))])
         self.h_meta = [pin((self.meta.nbytes,), torch.uint8) for _ in range(H)]
         self.d_meta = [torch.empty(self.meta.nbytes, dtype=torch.uint8, device=device) for _ in range(D2)]
         hv = [self.meta.views(b) for b in self.h_meta]
         dv = [self.meta.views(b) for b in self.d_meta]
-        self.h_tables, self.h_lens, self.h_slots, self.h_cow, self.h_pslots = (
-            [v[k] for v in hv] for k in ("tables", "lens", "slots", "cow", "pslots"))
-        self.d_tables, self.d_lens, self.d_slots, self.d_cow, self.d_pslots = (
-            [v[k] for v in dv] for k in ("tables", "lens", "slots", "cow", "pslots"))
+        self.h_tables, self.h_lens, self.h_cow, self.h_all_slots = (
+            [v[k] for v in hv] for k in ("tables", "lens", "cow", "slots"))
+        self.d_tables, self.d_lens, self.d_cow, self.d_slots = (
+            [v[k] for v in dv] for k in ("tables", "lens", "cow", "slots"))
+        self.h_slots = [x[:n] for x in self.h_all_slots]      # token slots
+        self.h_pslots = [x[n:] for x in self.h_all_slots]     # admitted prompts' slots
         self.h_done = [None] * H
         self.d_free = [None] * D2
         if e2e_from is not None:
@@ -464,7 +467,7 @@ class Replica:
         # 3. uploads (metadata; end to end also the step's inputs) on the copy stream
         if self.d_free[ds] is not None:
             self.copy.wait_event(self.d_free[ds])
-        mbytes = self.meta.off["pslots"] + ptot * 8          # everything through the used prompt slots
+        mbytes = self.meta.off["slots"] + (n + ptot) * 8     # everything through the used slots
         h2d = mbytes
         with torch.cuda.stream(self.copy):
             self.d_meta[ds][:mbytes].copy_(self.h_meta[hs][:mbytes], non_blocking=True)
@@ -475,8 +478,7 @@ class Replica:
                     self.d_in[ds][layer][:nb].copy_(host[:nb], non_blocking=True)
                     h2d += nb
                     v = self.e2e_views[t][layer]
-                    assert v["pk"].shape[0] == ptot
-                    layers.append((v["q"], v["k"], v["v"], v["pk"] if ptot else None, v["pv"] if ptot else None))
+                    layers.append((v["q"], v["k"], v["v"]))
             else:
                 layers = self.inputs[t]
             up = torch.cuda.Event()
@@ -490,10 +492,10 @@ class Replica:
             self.flush.fill_(t & 0xFF)
         if ncow:
             pa.pa_copy_blocks(self.cache.pool, self.d_cow[ds], ncow, stream=self.compute)
-        for layer, (q, k, v, pk, pv) in enumerate(layers):
-            if ptot:
-                pa.pa_append_kv(self.cache.pool, layer, pk, pv, self.d_pslots[ds], ptot, stream=self.compute)
-            pa.pa_append_kv(self.cache.pool, layer, k, v, self.d_slots[ds], n, stream=self.compute)
+        for layer, (q, k, v) in enumerate(layers):
+            # one launch appends the token rows and the admitted prompts' rows
+            assert k.shape[0] == n + ptot
+            pa.pa_append_kv(self.cache.pool, layer, k, v, self.d_slots[ds], n + ptot, stream=self.compute)
             if time_attention:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e0.record(self.compute)

@@ -1,5 +1,6 @@
 """Host-side staging of bench.py on CPU: the packed layouts that let one copy upload a
-step's metadata (and, end to end, a layer's q/K/V and prompt rows)."""
+step's metadata (and, end to end, a layer's q and K / V rows), and one append launch write
+the step's token rows and its admitted prompts' rows."""
 import numpy as np
 import pytest
 import torch
@@ -7,10 +8,13 @@ import torch
 import bench
 
 
-def _meta(n=5, mb=7, max_prompt=11):
+N = 5
+
+
+def _meta(n=N, mb=7, max_prompt=11):
+    # the benchmark's layout: slots last, the n token slots then the prompt slots
     return bench.Packed([("tables", torch.int32, (n, mb)), ("lens", torch.int32, (n,)),
-                         ("slots", torch.int64, (n,)), ("cow", torch.int32, (n, 2)),
-                         ("pslots", torch.int64, (max_prompt,))])
+                         ("cow", torch.int32, (n, 2)), ("slots", torch.int64, (n + max_prompt,))])
 
 
 def test_parts_are_aligned_disjoint_and_in_order():
@@ -28,11 +32,23 @@ def test_views_have_the_part_shapes_and_write_through():
     buf = torch.zeros(m.nbytes, dtype=torch.uint8)
     v = m.views(buf)
     assert v["tables"].shape == (5, 7) and v["tables"].dtype == torch.int32 and v["tables"].is_contiguous()
-    assert v["cow"].shape == (5, 2) and v["pslots"].dtype == torch.int64
+    assert v["cow"].shape == (5, 2) and v["slots"].dtype == torch.int64 and v["slots"].shape == (5 + 11,)
     v["tables"][:] = torch.arange(35, dtype=torch.int32).view(5, 7)
-    v["pslots"][:3] = torch.tensor([7, -1, 1 << 40])
+    v["slots"][N:N + 3] = torch.tensor([7, -1, 1 << 40])
     w = m.views(buf.clone())
-    assert torch.equal(w["tables"], v["tables"]) and w["pslots"][:3].tolist() == [7, -1, 1 << 40]
+    assert torch.equal(w["tables"], v["tables"]) and w["slots"][N:N + 3].tolist() == [7, -1, 1 << 40]
+
+
+def test_token_and_prompt_slots_are_one_run():
+    """The step reserves the prompts' slots into slots[n:] and the token slots into
+    slots[:n]; the append launch then reads slots[:n + ptot] in the order of its rows."""
+    m = _meta()
+    v = m.views(torch.zeros(m.nbytes, dtype=torch.uint8))
+    tok, prm = v["slots"][:N], v["slots"][N:]
+    tok.copy_(torch.arange(100, 100 + N))
+    prm[:4].copy_(torch.tensor([3, 4, 5, 6]))
+    assert v["slots"][:N + 4].tolist() == list(range(100, 100 + N)) + [3, 4, 5, 6]
+    assert tok.data_ptr() + N * 8 == prm.data_ptr()
 
 
 def test_one_prefix_copy_carries_every_part_and_the_used_prompt_slots():
@@ -40,27 +56,27 @@ def test_one_prefix_copy_carries_every_part_and_the_used_prompt_slots():
     host = torch.zeros(m.nbytes, dtype=torch.uint8)
     hv = m.views(host)
     rng = np.random.default_rng(0)
-    for name in ("tables", "lens", "slots", "cow", "pslots"):
+    for name in ("tables", "lens", "cow", "slots"):
         hv[name].copy_(torch.from_numpy(rng.integers(-9, 1 << 20, hv[name].shape).astype(
             np.int64 if hv[name].dtype == torch.int64 else np.int32)))
     ptot = 4
-    nb = m.off["pslots"] + ptot * 8
+    nb = m.off["slots"] + (N + ptot) * 8
     dev = torch.full((m.nbytes,), 0xEE, dtype=torch.uint8)
     dev[:nb].copy_(host[:nb])
     dv = m.views(dev)
-    for name in ("tables", "lens", "slots", "cow"):
+    for name in ("tables", "lens", "cow"):
         assert torch.equal(dv[name], hv[name])
-    assert torch.equal(dv["pslots"][:ptot], hv["pslots"][:ptot])
-    assert not torch.equal(dv["pslots"][ptot:], hv["pslots"][ptot:])   # unused slots were not copied
+    assert torch.equal(dv["slots"][:N + ptot], hv["slots"][:N + ptot])
+    assert not torch.equal(dv["slots"][N + ptot:], hv["slots"][N + ptot:])   # unused slots were not copied
 
 
-def test_empty_prompt_part():
-    p = bench.Packed([("q", torch.bfloat16, (4, 2, 8)), ("pk", torch.bfloat16, (0, 2, 8)),
-                      ("pv", torch.bfloat16, (0, 2, 8))])
+def test_empty_part():
+    p = bench.Packed([("q", torch.bfloat16, (4, 2, 8)), ("a", torch.bfloat16, (0, 2, 8)),
+                      ("b", torch.bfloat16, (0, 2, 8))])
     v = p.views(torch.zeros(p.nbytes, dtype=torch.uint8))
-    assert v["pk"].shape == (0, 2, 8) and v["pv"].numel() == 0
-    assert p.end["q"] == 4 * 2 * 8 * 2 and p.off["pk"] == bench.Packed.ALIGN
-    assert p.end["pv"] == p.off["pv"] == p.off["pk"]
+    assert v["a"].shape == (0, 2, 8) and v["b"].numel() == 0
+    assert p.end["q"] == 4 * 2 * 8 * 2 and p.off["a"] == bench.Packed.ALIGN
+    assert p.end["b"] == p.off["b"] == p.off["a"]
 
 
 @pytest.mark.parametrize("workload", ["large_pool_b16", "large_pool_b32", "prefix_sharing", "worked_example"])
