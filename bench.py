@@ -430,7 +430,15 @@ class Replica:
         self.readback = torch.cuda.Stream(device)
         self.scale = 1.0 / math.sqrt(sh.head_dim)
         self.attn_events = []
-        self.kv_bytes, self.alg_bytes, self.h2d, self.d2h, self.prompt_rows_appended = [], [], [], [], []
+        self._kv_bytes, self._alg_bytes, self.h2d, self.d2h, self.prompt_rows_appended = [], [], [], [], []
+        self._pending_lens = []   # each step's lengths, turned into byte counts off the step's path
+        # events are made once and re-recorded: per staging set the upload's, per device set
+        # the compute's and the read-back's, and a pair around each timed attention call
+        self.up_ev = [torch.cuda.Event() for _ in range(H)]
+        self.free_ev = [torch.cuda.Event() for _ in range(D2)]
+        self.rd_ev = [torch.cuda.Event() for _ in range(D2)]
+        self.attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                        for _ in range(total_steps * self.NL)]
         self.host_s = []
         self.flush = (torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device) if workload in L2_RESIDENT
                       else None)
@@ -481,7 +489,7 @@ class Replica:
                     layers.append((v["q"], v["k"], v["v"]))
             else:
                 layers = self.inputs[t]
-            up = torch.cuda.Event()
+            up = self.up_ev[hs]
             up.record(self.copy)
         self.h_done[hs] = up
         self.compute.wait_event(up)
@@ -497,15 +505,14 @@ class Replica:
             assert k.shape[0] == n + ptot
             pa.pa_append_kv(self.cache.pool, layer, k, v, self.d_slots[ds], n + ptot, stream=self.compute)
             if time_attention:
-                e0 = torch.cuda.Event(enable_timing=True)
+                e0, e1 = self.attn_ev[len(self.attn_events)]
                 e0.record(self.compute)
             pa.pa_decode_attention(self.cache.pool, layer, q, self.out[ds][layer], self.d_tables[ds],
                                    self.d_lens[ds], self.scale, self.split, self.ws, stream=self.compute)
             if time_attention:
-                e1 = torch.cuda.Event(enable_timing=True)
                 e1.record(self.compute)
                 self.attn_events.append((e0, e1))
-        free = torch.cuda.Event()
+        free = self.free_ev[ds]
         free.record(self.compute)
         self.d_free[ds] = free
         d2h = 0
@@ -513,25 +520,44 @@ class Replica:
             self.readback.wait_event(free)
             with torch.cuda.stream(self.readback):
                 self.h_out[ds].copy_(self.out[ds], non_blocking=True)
-                rd = torch.cuda.Event()
+                rd = self.rd_ev[ds]
                 rd.record(self.readback)
             self.out_read[ds] = rd
             d2h = self.out[ds].numel() * self.out[ds].element_size()
         # 5. retirements: blocks go back to the free list at once
         for slot, _ in plan["retire"]:
             self.cache.free(self.sids[slot])
-        # accounting: bytes decode attention reads / writes this step (all layers)
-        L = lens.numpy().astype(np.int64)
-        e = 2                                                  # bytes of a query / output element
-        row = sh.head_dim + 1 if self.kv_fp8 else sh.head_dim * e   # cached bytes of one (token, head) row
-        kv = self.NL * int((2 * L * sh.num_kv_heads * row).sum())
-        alg = kv + self.NL * (2 * n * sh.num_q_heads * sh.head_dim * e + int((4 * -(-L // sh.block_size)).sum())
-                              + 4 * n)
-        self.kv_bytes.append(kv)
-        self.alg_bytes.append(alg)
+        self._pending_lens.append(lens.numpy().copy())   # counted in _settle, off this path
         self.host_s.append(time.perf_counter() - h0)
         self.h2d.append(h2d)
         self.d2h.append(d2h)
+
+    def _settle(self):
+        """Bytes decode attention read / wrote in each step recorded since the last call
+        (all layers), from that step's sequence lengths."""
+        sh, n = self.shape, self.n
+        e = 2                                                  # bytes of a query / output element
+        row = sh.head_dim + 1 if self.kv_fp8 else sh.head_dim * e   # cached bytes of one (token, head) row
+        for lens in self._pending_lens:
+            L = lens.astype(np.int64)
+            kv = self.NL * int((2 * L * sh.num_kv_heads * row).sum())
+            alg = kv + self.NL * (2 * n * sh.num_q_heads * sh.head_dim * e +
+                                  int((4 * -(-L // sh.block_size)).sum()) + 4 * n)
+            self._kv_bytes.append(kv)
+            self._alg_bytes.append(alg)
+        self._pending_lens.clear()
+
+    @property
+    def kv_bytes(self):
+        """KV bytes decode attention read, per step so far."""
+        self._settle()
+        return self._kv_bytes
+
+    @property
+    def alg_bytes(self):
+        """Algorithmic bytes of decode attention (KV, q, out, tables, lengths), per step."""
+        self._settle()
+        return self._alg_bytes
 
     def drain(self):
         """Make the compute stream wait for outstanding read-backs (end of a timed leg)."""
