@@ -10,10 +10,10 @@ slot at the next step.  ``--workload`` selects the other synthetic workloads (th
 pages' worked example, prefix sharing, the ~100 GB 32-layer large pool with block
 16 or 32).
 
-A timed step runs the whole path: admissions (prompt K/V appended), one-slot
-reservations with the copy-on-write check (host, native), metadata upload, then for
-every layer the append of the step's K/V and decode attention (+ split-K reduce),
-and retirements (host).  Host bookkeeping of step t+1 overlaps the GPU work of step
+A timed step runs the whole path: admissions, one-slot reservations with the
+copy-on-write check (host, native), metadata upload, then for every layer one append
+of the step's K/V rows and the admitted prompts' rows, and decode attention (split
+ranges merged in the kernel), and retirements (host).  Host bookkeeping of step t+1 overlaps the GPU work of step
 t: metadata is staged in pinned buffers and uploaded on a side stream into
 NSETS rotating device buffer sets.
 
