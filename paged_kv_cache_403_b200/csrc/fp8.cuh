@@ -82,59 +82,103 @@ struct AppendParams {
     const int64_t *slots;
     int32_t n_tokens, block_size, num_kv_heads;
     int64_t num_blocks;
+    Div32 by_heads, by_block;       // num_kv_heads, block_size (32-bit index form)
 };
 
-// One warp per (token, head) row of K or V: amax by a warp max of the fp32 bit
-// patterns (non-negative floats order like their bits), the row exponent from the
-// bits of amax, one fp32 multiply by 2^-X per element, then E4M3 rounding.
-template <typename T, int D>
+// kAppendLanes lanes per (token, head) row of K or V, so a warp quantises 32 / kAppendLanes
+// rows at once and the per-row work (index arithmetic, slot check, the exponent) is shared
+// by lanes of D / kAppendLanes elements each -- with a warp per row the kernel was bound by
+// instruction issue, not memory.  amax by a max over the row's lanes of the fp32 bit
+// patterns (non-negative floats order like their bits), the row exponent from the bits of
+// amax, one fp32 multiply by 2^-X per element, then E4M3 rounding.  The rows of a warp may
+// take different paths (a padding slot, a bad slot), so every shuffle is executed by the
+// whole warp and only the stores are guarded.
+constexpr int kAppendLanes = 4;
+template <typename T, int D, bool NARROW>
 __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
-    constexpr int EPL = D / 32;   // elements per lane: 2 or 4
-    static_assert(EPL == 2 || EPL == 4, "head_dim 64 or 128");
+    constexpr int LPR = kAppendLanes, RPW = 32 / LPR;   // lanes per row, rows per warp
+    constexpr int EPL = D / LPR;                         // elements per lane: 8, 16 or 32
+    static_assert(EPL == 8 || EPL == 16 || EPL == 32, "head_dim 64 or 128");
+    constexpr int NQ = EPL / 8;                          // 16-byte loads per lane
     const int lane = threadIdx.x & 31;
+    const int rl = lane % LPR;                           // lane within the row
     const int64_t rows = (int64_t)p.n_tokens * p.num_kv_heads;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < 2 * rows; r += warps) {
+    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); RPW * w < 2 * rows; w += warps) {
+        const int64_t r = RPW * w + lane / LPR;           // this row: K rows, then V rows
+        bool valid = r < 2 * rows;
         const bool is_v = r >= rows;
         const int64_t rr = is_v ? r - rows : r;
-        const int64_t i = rr / p.num_kv_heads;
-        const int h = (int)(rr % p.num_kv_heads);
-        // the row is read before the slot is looked at, so the two loads overlap
-        const unsigned char *src = (is_v ? p.v_new : p.k_new) + (size_t)(rr * D + lane * EPL) * sizeof(T);
-        uint2 u;
-        if constexpr (EPL == 4)
-            u = *reinterpret_cast<const uint2 *>(src);
-        else
-            u.x = *reinterpret_cast<const uint32_t *>(src);
-        const int64_t slot = p.slots[i];
-        if (slot < 0) continue;
-        const int64_t blk = slot / p.block_size;
-        const int off = (int)(slot % p.block_size);
-        if (blk >= p.num_blocks) {
-            if (lane == 0 && !is_v) raise_error(kErrBadSlot);
-            continue;
+        int64_t i = 0;
+        int h = 0;
+        if (valid) {
+            if constexpr (NARROW) {   // 32-bit index arithmetic (see Div32)
+                i = div32((uint32_t)rr, p.by_heads);
+                h = (int)((uint32_t)rr - (uint32_t)i * (uint32_t)p.num_kv_heads);
+            } else {
+                i = rr / p.num_kv_heads;
+                h = (int)(rr % p.num_kv_heads);
+            }
         }
+        // the row is read before the slot is looked at, so the loads overlap
+        uint4 u[NQ] = {};
+        int64_t slot = -1;
+        if (valid) {
+            const uint4 *src = reinterpret_cast<const uint4 *>((is_v ? p.v_new : p.k_new) +
+                                                               (size_t)(rr * D + rl * EPL) * sizeof(T));
+#pragma unroll
+            for (int k = 0; k < NQ; ++k) u[k] = src[k];
+            slot = p.slots[i];
+        }
+        if (valid && slot >= p.num_blocks * p.block_size) {
+            if (rl == 0 && !is_v) raise_error(kErrBadSlot);
+            valid = false;
+        }
+        if (slot < 0) valid = false;             // padding row
         float x[EPL];
-        Elem<T>::widen2(u.x, x);
-        if constexpr (EPL == 4) Elem<T>::widen2(u.y, x + 2);
+#pragma unroll
+        for (int k = 0; k < NQ; ++k) {
+            Elem<T>::widen2(u[k].x, x + 8 * k);
+            Elem<T>::widen2(u[k].y, x + 8 * k + 2);
+            Elem<T>::widen2(u[k].z, x + 8 * k + 4);
+            Elem<T>::widen2(u[k].w, x + 8 * k + 6);
+        }
         uint32_t a = 0;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) a = max(a, __float_as_uint(x[e]) & 0x7fffffffu);
-        a = __reduce_max_sync(0xffffffffu, a);
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, o));   // within the row
+        if (!valid) continue;
+        int64_t blk;
+        int off;
+        if constexpr (NARROW) {
+            blk = div32((uint32_t)slot, p.by_block);
+            off = (int)((uint32_t)slot - (uint32_t)blk * (uint32_t)p.block_size);
+        } else {
+            blk = slot / p.block_size;
+            off = (int)(slot % p.block_size);
+        }
         // smallest X with amax <= 448 * 2^X: amax = 1.M * 2^(E-127) <= 1.75 * 2^(8+X)
         const int E = (int)(a >> 23);
         int X = E == 0 ? -127 : ((a & 0x7fffffu) <= 0x600000u ? E - 135 : E - 134);
         X = max(-127, min(127, X));
         const float f = __uint_as_float((uint32_t)(127 - X) << 23);   // 2^-X (127 - X >= 6)
-        uint32_t codes = f32x2_to_e4m3x2(x[0] * f, x[1] * f);
-        if constexpr (EPL == 4) codes |= f32x2_to_e4m3x2(x[2] * f, x[3] * f) << 16;
+        uint32_t codes[EPL / 4];
+#pragma unroll
+        for (int k = 0; k < EPL / 4; ++k)
+            codes[k] = f32x2_to_e4m3x2(x[4 * k] * f, x[4 * k + 1] * f) |
+                       (f32x2_to_e4m3x2(x[4 * k + 2] * f, x[4 * k + 3] * f) << 16);
         const size_t row = ((size_t)blk * p.num_kv_heads + h) * p.block_size + off;
-        unsigned char *dst = (is_v ? p.v_layer : p.k_layer) + row * D + lane * EPL;
-        if constexpr (EPL == 4)
-            *reinterpret_cast<uint32_t *>(dst) = codes;
-        else
-            *reinterpret_cast<uint16_t *>(dst) = (uint16_t)codes;
-        if (lane == 0)
+        unsigned char *dst = (is_v ? p.v_layer : p.k_layer) + row * D + rl * EPL;
+        if constexpr (EPL >= 16) {
+#pragma unroll
+            for (int k = 0; k < EPL / 16; ++k)
+                reinterpret_cast<uint4 *>(dst)[k] =
+                    make_uint4(codes[4 * k], codes[4 * k + 1], codes[4 * k + 2], codes[4 * k + 3]);
+        } else {
+            *reinterpret_cast<uint2 *>(dst) = make_uint2(codes[0], codes[1]);
+        }
+        if (rl == 0)
             p.s_layer[(((size_t)blk * p.num_kv_heads + h) * 2 + (is_v ? 1 : 0)) * p.block_size + off] =
                 (unsigned char)(X + 127);
     }

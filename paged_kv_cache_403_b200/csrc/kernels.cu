@@ -51,6 +51,19 @@ __device__ unsigned int g_device_error = 0;
 
 __device__ __forceinline__ void raise_error(unsigned e) { atomicOr(&g_device_error, e); }
 
+// Division of 32-bit indices by a divisor fixed for the launch: a shift when it is a power
+// of two, else the hardware's 32-bit division.  The append kernels' index arithmetic in 64
+// bits (emulated division) cost more than their memory traffic; the host launches the
+// 32-bit form only when every index of the launch fits.
+struct Div32 {
+    uint32_t d;
+    int32_t shift;   // >= 0: d == 1 << shift
+};
+inline Div32 make_div32(uint32_t d) {
+    return {d, (d && !(d & (d - 1))) ? __builtin_ctz(d) : -1};
+}
+__device__ __forceinline__ uint32_t div32(uint32_t n, Div32 d) { return d.shift >= 0 ? n >> d.shift : n / d.d; }
+
 // ------------------------------------------------------------------ PTX wrappers
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -1154,29 +1167,50 @@ struct AppendParams {
     const int64_t *slots;
     int32_t n_tokens, block_size, num_kv_heads, row_chunks;   // row_chunks = D*e/16
     int64_t num_blocks;
+    Div32 by_chunks, by_block, by_row_chunks;                 // Hkv*row_chunks, block_size, row_chunks
 };
 
 // One thread per 16-byte chunk of a new row (all tokens, heads and chunks flattened,
 // grid-stride); the source read is issued before the slot lookup, so a thread's loads
 // are in flight together.
+template <bool NARROW>
 __global__ void __launch_bounds__(256) append_kv_kernel(const AppendParams p) {
     const int64_t chunks = (int64_t)p.num_kv_heads * p.row_chunks;   // 16-byte chunks per token
     const int64_t total = (int64_t)p.n_tokens * chunks;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total; g += stride) {
-        const int64_t i = g / chunks;
-        const int t = (int)(g - i * chunks);
+        int64_t i;
+        int t;
+        if constexpr (NARROW) {
+            i = div32((uint32_t)g, p.by_chunks);
+            t = (int)((uint32_t)g - (uint32_t)i * (uint32_t)chunks);
+        } else {
+            i = g / chunks;
+            t = (int)(g - i * chunks);
+        }
         const uint4 kx = reinterpret_cast<const uint4 *>(p.k_new)[g];   // [n][Hkv][row_chunks]
         const uint4 vx = reinterpret_cast<const uint4 *>(p.v_new)[g];
         const int64_t slot = p.slots[i];
         if (slot < 0) continue;                                            // padding row
-        const int64_t blk = slot / p.block_size;
-        const int off = (int)(slot % p.block_size);
-        if (blk >= p.num_blocks) {
-            if (t == 0) raise_error(kErrBadSlot);
-            continue;
+        int64_t blk;
+        int off, h;
+        if constexpr (NARROW) {
+            if (slot >= p.num_blocks * p.block_size) {
+                if (t == 0) raise_error(kErrBadSlot);
+                continue;
+            }
+            blk = div32((uint32_t)slot, p.by_block);
+            off = (int)((uint32_t)slot - (uint32_t)blk * (uint32_t)p.block_size);
+            h = (int)div32((uint32_t)t, p.by_row_chunks);
+        } else {
+            blk = slot / p.block_size;
+            off = (int)(slot % p.block_size);
+            if (blk >= p.num_blocks) {
+                if (t == 0) raise_error(kErrBadSlot);
+                continue;
+            }
+            h = t / p.row_chunks;
         }
-        const int h = t / p.row_chunks;
         const int c = t - h * p.row_chunks;
         const size_t dst = (((size_t)blk * p.num_kv_heads + h) * p.block_size + off) * p.row_chunks + c;
         reinterpret_cast<uint4 *>(p.k_layer)[dst] = kx;
@@ -1758,21 +1792,29 @@ pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const vo
         p.block_size = c.block_size;
         p.num_kv_heads = c.num_kv_heads;
         p.num_blocks = c.num_blocks;
-        const int64_t warps = 2 * (int64_t)n_tokens * c.num_kv_heads;
+        const int64_t rows2 = 2 * (int64_t)n_tokens * c.num_kv_heads;   // K rows, then V rows
+        const int64_t warps = (rows2 + 32 / fp8::kAppendLanes - 1) / (32 / fp8::kAppendLanes);
         const int grid = (int)std::min<int64_t>((warps + 7) / 8, 148 * 16);
+        p.by_heads = make_div32((uint32_t)c.num_kv_heads);
+        p.by_block = make_div32((uint32_t)c.block_size);
+        const bool narrow = rows2 < INT32_MAX && (int64_t)c.num_blocks * c.block_size < INT32_MAX;
         cudaStream_t cs = static_cast<cudaStream_t>(stream);
         const bool bf = c.act_dtype == PA_BF16;
+#define PA_FP8_APPEND(TT, DD)                                                          \
+    (narrow ? fp8::append_kernel<TT, DD, true><<<grid, 256, 0, cs>>>(p)              \
+            : fp8::append_kernel<TT, DD, false><<<grid, 256, 0, cs>>>(p))
         if (c.head_dim == 128) {
             if (bf)
-                fp8::append_kernel<__nv_bfloat16, 128><<<grid, 256, 0, cs>>>(p);
+                PA_FP8_APPEND(__nv_bfloat16, 128);
             else
-                fp8::append_kernel<__half, 128><<<grid, 256, 0, cs>>>(p);
+                PA_FP8_APPEND(__half, 128);
         } else {
             if (bf)
-                fp8::append_kernel<__nv_bfloat16, 64><<<grid, 256, 0, cs>>>(p);
+                PA_FP8_APPEND(__nv_bfloat16, 64);
             else
-                fp8::append_kernel<__half, 64><<<grid, 256, 0, cs>>>(p);
+                PA_FP8_APPEND(__half, 64);
         }
+#undef PA_FP8_APPEND
         pa_internal::launch_count.fetch_add(1);
         return check_launch("fp8::append_kernel");
     }
@@ -1791,7 +1833,14 @@ pa_status pa_append_kv(pa_pool *pool, int32_t layer, const void *k_new, const vo
     p.num_blocks = pool->cfg.num_blocks;
     const int64_t threads = (int64_t)n_tokens * p.num_kv_heads * p.row_chunks;
     const int grid = (int)std::min<int64_t>((threads + 255) / 256, 148 * 16);
-    append_kv_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    p.by_chunks = make_div32((uint32_t)(p.num_kv_heads * p.row_chunks));
+    p.by_block = make_div32((uint32_t)p.block_size);
+    p.by_row_chunks = make_div32((uint32_t)p.row_chunks);
+    const bool narrow = threads < INT32_MAX && p.num_blocks * p.block_size < INT32_MAX;
+    if (narrow)
+        append_kv_kernel<true><<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    else
+        append_kv_kernel<false><<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
     pa_internal::launch_count.fetch_add(1);
     return check_launch("append_kv_kernel");
 }
